@@ -1,0 +1,359 @@
+"""Float64 CPU oracle for Looped Latent Attention (LLA) decode.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports this module; only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` call
+it.  It shares no code with the CUDA path: plain NumPy in float64, written from
+the method's definition so that a reader can check each step against the pages.
+
+Pages this follows (cited by page title and section):
+
+* [CR]  "Looped Latent Attention: 跨循环 KV 压缩精读" (cc.laoqi.cc close reading of
+        arXiv 2607.15456v2).  §二.1 symbol table, §二.2 eq. (4) and its worked
+        example, §二.3 pre-RoPE compression, §二.4 SVD initialisation,
+        §二.6 LLA-2D, §四.9 Table 5 (serving).
+* [GS]  "Looped Latent Attention: Cross-Loop KV Compression for Looped
+        Transformers" (gist.science explainer), "Technisches Resümee":
+        "Kernmechanismus" (encode / loop-specific decode formulas, LLA-2D),
+        "Zentrale Beiträge" (ratio formula), "Training und Initialisierung".
+* [PN]  daiwk Q&A digest, entry on RoPE pairing for Llama-family models
+        (split-half pairing), background for the RoPE layout reading.
+
+Conventions (row vectors throughout, as on [GS] Kernmechanismus):
+  per-head  x = [x_0; ...; x_{T-1}] in R^{T d}, loop-major, 0-based loops.
+  LLA-2D    x = concat over (t, h, i) in R^{T H d}, loop-major then head.
+  encode    c   = (x - mu) W_down,              W_down in R^{(T d) x r}
+  decode    x^_t = c W_up,t^T + mu_t,           W_up,t in R^{d x r}
+  RoPE      split-half: pair (i, i + d/2) rotated by angle pos * base^(-2i/d).
+
+Readings where the pages are silent are listed in the design notes; the ones
+that change arithmetic are restated next to the function that takes them.
+Every function here is pinned by ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from fractions import Fraction
+
+import numpy as np
+
+MODE_PER_HEAD = 0
+MODE_2D = 1
+
+
+@dataclass(frozen=True)
+class Cfg:
+    """Codec geometry.  [CR §二.1]: T loops, H heads, d_head, latent widths r_k, r_v."""
+
+    T: int
+    H: int
+    d: int
+    r_k: int
+    r_v: int
+    mode: int = MODE_PER_HEAD
+    rope_base: float = 10000.0
+
+    @property
+    def width(self) -> int:
+        """Width of the concatenated trajectory that one latent encodes."""
+        return self.T * self.d if self.mode == MODE_PER_HEAD else self.T * self.H * self.d
+
+
+# --------------------------------------------------------------------------
+# bf16 rounding (the cache number format).  Round-to-nearest-even from float64.
+# --------------------------------------------------------------------------
+
+def bf16_round(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (ties to even), return float64.
+
+    bfloat16 = 1 sign, 8 exponent, 7 stored mantissa bits (8 significant bits).
+    Normal numbers keep 8 significant bits; below 2^-126 the spacing is fixed at
+    2^-133 (subnormals).  Values past the largest finite bf16 plus half an ulp
+    become +-inf.  Rounding happens once, straight from float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    finite = np.isfinite(x)
+    out[~finite] = x[~finite]
+    xf = x[finite]
+    m, e = np.frexp(xf)                       # xf = m * 2^e, 0.5 <= |m| < 1
+    normal = e >= -125                        # |x| >= 2^-126
+    q = np.where(normal, np.ldexp(np.rint(np.ldexp(m, 8)), e - 8),
+                 np.ldexp(np.rint(np.ldexp(xf, 133)), -133))
+    max_bf16 = np.ldexp(255.0, 127 - 7)       # (2 - 2^-7) * 2^127
+    q = np.where(np.abs(q) > max_bf16, np.copysign(np.inf, xf), q)
+    out[finite] = q
+    return out
+
+
+# --------------------------------------------------------------------------
+# Bookkeeping: exact cache sizes and ratio  ([CR §二.2 eq. (4)], [GS Zentrale Beiträge])
+# --------------------------------------------------------------------------
+
+def teacher_scalars_per_token_layer(cfg: Cfg) -> int:
+    """Uncompressed loop-indexed cache: K and V for every loop and head: 2 T H d."""
+    return 2 * cfg.T * cfg.H * cfg.d
+
+
+def lla_scalars_per_token_layer(cfg: Cfg) -> int:
+    """LLA cache: (r_k + r_v) per head, H heads; LLA-2D stores r_k + r_v in total [CR §二.6]."""
+    per = cfg.r_k + cfg.r_v
+    return per * cfg.H if cfg.mode == MODE_PER_HEAD else per
+
+
+def compression_ratio(cfg: Cfg) -> Fraction:
+    """Exact ratio of persistent cache scalars at equal precision.
+
+    Per head this is 2 T d_head / (r_k + r_v) ([GS Zentrale Beiträge], [CR eq. (4)]);
+    for LLA-2D it is 2 T H d / (r_k + r_v).
+    """
+    return Fraction(teacher_scalars_per_token_layer(cfg), lla_scalars_per_token_layer(cfg))
+
+
+def cache_bytes(cfg: Cfg, tokens: int, layers: int, bytes_per_scalar: int = 2) -> int:
+    """Persistent latent-cache bytes for ``tokens`` tokens over ``layers`` shared layers."""
+    return lla_scalars_per_token_layer(cfg) * tokens * layers * bytes_per_scalar
+
+
+def teacher_cache_bytes(cfg: Cfg, tokens: int, layers: int, bytes_per_scalar: int = 2) -> int:
+    return teacher_scalars_per_token_layer(cfg) * tokens * layers * bytes_per_scalar
+
+
+# --------------------------------------------------------------------------
+# Codec: encode / loop-specific decode ([GS Kernmechanismus], [CR §二.1])
+# --------------------------------------------------------------------------
+
+def encode(x: np.ndarray, mu: np.ndarray, W_down: np.ndarray) -> np.ndarray:
+    """c = (x - mu) W_down.  x: [..., W] concatenated trajectory, mu: [W], W_down: [W, r]."""
+    x = np.asarray(x, dtype=np.float64)
+    return (x - np.asarray(mu, dtype=np.float64)) @ np.asarray(W_down, dtype=np.float64)
+
+
+def reconstruct(c: np.ndarray, W_up_t: np.ndarray, mu_t: np.ndarray) -> np.ndarray:
+    """x^_t = c W_up,t^T + mu_t.  c: [..., r], W_up_t: [d, r], mu_t: [d]."""
+    c = np.asarray(c, dtype=np.float64)
+    return c @ np.asarray(W_up_t, dtype=np.float64).T + np.asarray(mu_t, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# RoPE, split-half layout ([CR §二.3]: applied after reconstruction, full dimension)
+# --------------------------------------------------------------------------
+
+def rope_inv_freq(d: int, base: float) -> np.ndarray:
+    """theta_i = base^(-2 i / d) for i < d/2, in float64."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * i / d)
+
+
+def rope(x: np.ndarray, pos, base: float) -> np.ndarray:
+    """Rotate pair (x_i, x_{i+d/2}) by angle pos * theta_i.
+
+    x: [..., d]; pos: integer array broadcastable to x.shape[:-1].
+    Angles are formed in float64 (reading: the pages fix no RoPE precision).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    h = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_inv_freq(d, base)
+    cos, sin = np.cos(ang), np.sin(ang)
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * cos - b * sin, a * sin + b * cos], axis=-1)
+
+
+# --------------------------------------------------------------------------
+# Attention for one query (decode) over a history plus the in-flight token
+# --------------------------------------------------------------------------
+
+def attention_plain(q, K_hist, V_hist, pos_hist, k_self, v_self, q_pos, base, scale=None):
+    """Decode attention over an uncompressed per-loop cache.
+
+    q, k_self, v_self: [d] pre-RoPE; K_hist, V_hist: [n, d] pre-RoPE; pos_hist: [n].
+    Scores s = RoPE(q, q_pos) . RoPE(k, pos) * scale over the history and the
+    in-flight token (at q_pos); softmax with max subtraction; output sum p v.
+    Returns (out [d], p_hist [n], p_self).
+    """
+    q = np.asarray(q, np.float64)
+    d = q.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    K_hist = np.asarray(K_hist, np.float64).reshape(-1, d)
+    V_hist = np.asarray(V_hist, np.float64).reshape(-1, d)
+    qr = rope(q, q_pos, base)
+    kr = rope(K_hist, np.asarray(pos_hist), base)
+    ks = rope(np.asarray(k_self, np.float64), q_pos, base)
+    s = np.concatenate([kr @ qr, [ks @ qr]]) * scale
+    s = s - s.max()
+    p = np.exp(s)
+    p = p / p.sum()
+    out = p[:-1] @ V_hist + p[-1] * np.asarray(v_self, np.float64)
+    return out, p[:-1], p[-1]
+
+
+def decode_attention(q, k_self, v_self, c_k, c_v, W_up_k_t, W_up_v_t, mu_k_t, mu_v_t,
+                     positions, q_pos, base, scale=None):
+    """LLA decode attention at loop t, direct form.
+
+    Rebuild loop t's history K and V from the latents ([GS Kernmechanismus]),
+    then attend as ``attention_plain``.  The in-flight token's loop-t K/V is exact
+    (it is encoded only after its last loop).  Returns out [d].
+    """
+    K = reconstruct(c_k, W_up_k_t, mu_k_t)
+    V = reconstruct(c_v, W_up_v_t, mu_v_t)
+    out, _, _ = attention_plain(q, K, V, positions, k_self, v_self, q_pos, base, scale)
+    return out
+
+
+def decode_attention_absorbed(q, k_self, v_self, c_k, c_v, W_up_k_t, W_up_v_t, mu_k_t, mu_v_t,
+                              positions, q_pos, base, scale=None):
+    """Same result with V never rebuilt per token.
+
+    Because the weights p sum to one over history plus self,
+      sum_j p_j (c_v,j W^T + mu) + p_self v_self
+        = (sum_j p_j c_v,j) W^T + (sum_j p_j) mu + p_self v_self,
+    so values are summed in latent space and up-projected once.
+    """
+    K = reconstruct(c_k, W_up_k_t, mu_k_t)
+    d = np.asarray(q).shape[-1]
+    zeros = np.zeros((K.shape[0], d))
+    _, p_hist, p_self = attention_plain(q, K, zeros, positions, k_self, np.zeros(d), q_pos,
+                                        base, scale)
+    W_up_v_t = np.asarray(W_up_v_t, np.float64)
+    c_v = np.asarray(c_v, np.float64).reshape(K.shape[0], W_up_v_t.shape[1])
+    o_lat = p_hist @ c_v
+    return (o_lat @ W_up_v_t.T
+            + p_hist.sum() * np.asarray(mu_v_t, np.float64)
+            + p_self * np.asarray(v_self, np.float64))
+
+
+# --------------------------------------------------------------------------
+# Whole-cache wrappers with the library's data layout (used by parity tests)
+# --------------------------------------------------------------------------
+
+@dataclass
+class Codec:
+    """fp64 codec parameters.
+
+    per-head: W_down_[kv] [H, T*d, r], W_up_[kv] [H, T, d, r], mu_[kv] [H, T*d]
+    LLA-2D:   W_down_[kv] [T*H*d, r],  W_up_[kv] [T, H, d, r], mu_[kv] [T*H*d]
+    """
+
+    W_down_k: np.ndarray
+    W_down_v: np.ndarray
+    W_up_k: np.ndarray
+    W_up_v: np.ndarray
+    mu_k: np.ndarray
+    mu_v: np.ndarray
+
+
+def w_up_t(cfg: Cfg, W_up: np.ndarray, t: int, h: int) -> np.ndarray:
+    return W_up[h, t] if cfg.mode == MODE_PER_HEAD else W_up[t, h]
+
+
+def mu_t(cfg: Cfg, mu: np.ndarray, t: int, h: int) -> np.ndarray:
+    """Loop-t (and head-h) slice of the concatenated mean."""
+    d = cfg.d
+    if cfg.mode == MODE_PER_HEAD:
+        return mu[h, t * d:(t + 1) * d]
+    off = (t * cfg.H + h) * d
+    return mu[off:off + d]
+
+
+def encode_tokens(cfg: Cfg, codec: Codec, x_k, x_v):
+    """Encode finished tokens.  x_[kv]: [N, T, H, d] (per-loop K/V rows of each token).
+
+    Returns unrounded latents: per-head [N, H, r], LLA-2D [N, r].
+    """
+    x_k = np.asarray(x_k, np.float64)
+    x_v = np.asarray(x_v, np.float64)
+    N = x_k.shape[0]
+    if cfg.mode == MODE_PER_HEAD:
+        ck = np.empty((N, cfg.H, cfg.r_k))
+        cv = np.empty((N, cfg.H, cfg.r_v))
+        for h in range(cfg.H):
+            xk = x_k[:, :, h, :].reshape(N, cfg.T * cfg.d)    # loop-major concat
+            xv = x_v[:, :, h, :].reshape(N, cfg.T * cfg.d)
+            ck[:, h] = encode(xk, codec.mu_k[h], codec.W_down_k[h])
+            cv[:, h] = encode(xv, codec.mu_v[h], codec.W_down_v[h])
+        return ck, cv
+    xk = x_k.reshape(N, -1)                                     # (t, h, i) order
+    xv = x_v.reshape(N, -1)
+    return encode(xk, codec.mu_k, codec.W_down_k), encode(xv, codec.mu_v, codec.W_down_v)
+
+
+def decode_attn_cache(cfg: Cfg, codec: Codec, t: int, q, k_self, v_self, c_k, c_v,
+                      positions, q_pos, ctx_len, pairs=None, scale=None, absorbed=False):
+    """Decode attention for a batch, library layout.
+
+    q, k_self, v_self: [B, H, d]; c_k: per-head [B, n_cap, H, r_k], 2D [B, n_cap, r_k];
+    positions: [B, n_cap]; q_pos, ctx_len: [B].  ``pairs`` restricts the work to a
+    list of (b, h); the result holds NaN elsewhere.  Returns out [B, H, d].
+    """
+    q = np.asarray(q, np.float64)
+    B, H, d = q.shape
+    out = np.full((B, H, d), np.nan)
+    if pairs is None:
+        pairs = [(b, h) for b in range(B) for h in range(H)]
+    fn = decode_attention_absorbed if absorbed else decode_attention
+    for b, h in pairs:
+        n = int(ctx_len[b])
+        if cfg.mode == MODE_PER_HEAD:
+            ck = np.asarray(c_k[b, :n, h], np.float64)
+            cv = np.asarray(c_v[b, :n, h], np.float64)
+        else:
+            ck = np.asarray(c_k[b, :n], np.float64)
+            cv = np.asarray(c_v[b, :n], np.float64)
+        out[b, h] = fn(q[b, h], k_self[b, h], v_self[b, h], ck, cv,
+                       w_up_t(cfg, codec.W_up_k, t, h), w_up_t(cfg, codec.W_up_v, t, h),
+                       mu_t(cfg, codec.mu_k, t, h), mu_t(cfg, codec.mu_v, t, h),
+                       np.asarray(positions[b, :n]), int(q_pos[b]), cfg.rope_base, scale)
+    return out
+
+
+# --------------------------------------------------------------------------
+# SVD initialisation ([CR §二.4], [GS Training und Initialisierung])
+# --------------------------------------------------------------------------
+
+def svd_init(X: np.ndarray, r: int):
+    """Codec from calibration rows X [N, W] (concatenated trajectories).
+
+    mu = column mean; W_down = top-r right singular vectors of X - mu, ordered by
+    singular value.  Sign reading: each column's entry of largest magnitude is
+    made positive (the pages fix no sign).  Returns (mu [W], W_down [W, r], sigma).
+    """
+    X = np.asarray(X, np.float64)
+    mu = X.mean(axis=0)
+    _, sigma, Vt = np.linalg.svd(X - mu, full_matrices=False)
+    W = Vt[:r].T.copy()
+    idx = np.argmax(np.abs(W), axis=0)
+    sgn = np.sign(W[idx, np.arange(W.shape[1])])
+    sgn[sgn == 0] = 1.0
+    return mu, W * sgn, sigma
+
+
+def loop_slices(W_down: np.ndarray, T: int, d: int, H: int | None = None) -> np.ndarray:
+    """W_up,t initialised as the loop-t rows of W_down ([CR §二.4]).
+
+    per-head: returns [T, d, r]; LLA-2D (H given): returns [T, H, d, r].
+    """
+    r = W_down.shape[1]
+    if H is None:
+        return W_down.reshape(T, d, r).copy()
+    return W_down.reshape(T, H, d, r).copy()
+
+
+def svd_codec(cfg: Cfg, calib_k: np.ndarray, calib_v: np.ndarray) -> Codec:
+    """Build a full codec by SVD from calibration tokens calib_[kv]: [N, T, H, d]."""
+    N = calib_k.shape[0]
+    if cfg.mode == MODE_PER_HEAD:
+        parts = {"k": ([], [], []), "v": ([], [], [])}
+        for key, X, r in (("k", calib_k, cfg.r_k), ("v", calib_v, cfg.r_v)):
+            for h in range(cfg.H):
+                mu, Wd, _ = svd_init(X[:, :, h, :].reshape(N, cfg.T * cfg.d), r)
+                parts[key][0].append(Wd)
+                parts[key][1].append(loop_slices(Wd, cfg.T, cfg.d))
+                parts[key][2].append(mu)
+        return Codec(np.stack(parts["k"][0]), np.stack(parts["v"][0]),
+                     np.stack(parts["k"][1]), np.stack(parts["v"][1]),
+                     np.stack(parts["k"][2]), np.stack(parts["v"][2]))
+    mk, Wk, _ = svd_init(calib_k.reshape(N, -1), cfg.r_k)
+    mv, Wv, _ = svd_init(calib_v.reshape(N, -1), cfg.r_v)
+    return Codec(Wk, Wv, loop_slices(Wk, cfg.T, cfg.d, cfg.H), loop_slices(Wv, cfg.T, cfg.d, cfg.H),
+                 mk, mv)
