@@ -1,0 +1,405 @@
+"""Benchmark of the LLA decode hot path on B200.
+
+One step = one decode step of the workload: decode attention at each listed loop
+t over every layer's latent cache, then encode of the finished tokens (the
+per-loop K/V of the token that just completed its last loop).  Default workload:
+per-head LLA at 4x (T=4, H=16, d=128, r_k=96, r_v=160), batch 8, 4096-token
+context, one layer.
+
+Prints one JSON line (rank 0).  `value` is algorithmic HBM GB/s over the whole
+step with inputs resident in HBM; `e2e` is the same metric with the step's
+inputs copied from pinned host memory and the outputs read back inside the
+timed region.  `--impl reference` times the float64 CPU oracle on a bounded
+sample of the same workload (the reference arm of this benchmark).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = synth.WORKLOAD_ORDER[1]
+METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop step"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="lla", choices=["lla", "reference"])
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- byte counts
+
+def decode_bytes(w, n_ctx: int) -> int:
+    """Algorithmic HBM bytes of one decode call (one layer, one loop)."""
+    L = w.H if w.mode == synth.MODE_PER_HEAD else 1
+    lat = w.B * n_ctx * (w.r_k + w.r_v) * 2 * L
+    pos = w.B * n_ctx * 4
+    weights = w.H * w.d * (w.r_k + w.r_v) * 4 + 2 * w.H * w.d * 4
+    io = 4 * w.B * w.H * w.d * 4
+    return lat + pos + weights + io
+
+
+def encode_bytes(w, n_tok: int) -> int:
+    L = w.H if w.mode == synth.MODE_PER_HEAD else 1
+    width = w.T * w.d * (1 if L > 1 else w.H)
+    x = n_tok * w.T * w.H * w.d * 2 * 2
+    wd = L * (w.r_k + w.r_v) * width * 2 + L * (w.r_k + w.r_v) * 4
+    out = n_tok * L * (w.r_k + w.r_v) * 2 + n_tok * 8
+    return x + wd + out
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-i", str(gpu_index), "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        self.p.wait(timeout=10)
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def build_state(w, device):
+    import torch
+    import looped_transformer_decode_b200 as lla
+
+    cfg = lla.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
+    append = w.encode_tokens < w.B * w.n          # decode-time append: one new row per sequence
+    n_cap = w.n + 1 if append else w.n
+    layers = []
+    for layer in range(w.layers):
+        cod = synth.workload_codec(w, seed_offset=layer)
+        packed = lla.codec_pack(cfg, *(torch.from_numpy(cod[k]).to(device) for k in
+                                       ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
+        x = synth.workload_tensors(w, device, seed_offset=layer, n=n_cap)
+        x["ctx_len"].fill_(w.n)
+        x["q_pos"].fill_(w.n)
+        layers.append({"packed": packed, **x})
+    rope = lla.rope_table(cfg, n_cap + 1)
+    ws = lla.decode_workspace(cfg, w.B, n_cap)
+    n_tok = w.encode_tokens
+    xk, xv = synth.encode_inputs(w, device, n_tok)
+    if append:
+        slot = torch.arange(w.B, device=device, dtype=torch.int64) * n_cap + w.n
+    else:
+        slot = torch.arange(n_tok, device=device, dtype=torch.int64)
+    out = torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=device)
+    return {"cfg": cfg, "layers": layers, "rope": rope, "ws": ws, "xk": xk, "xv": xv,
+            "slot": slot, "out": out, "n_cap": n_cap}
+
+
+def run_step(lla, w, st, events=None):
+    for t in w.loops:
+        for L in st["layers"]:
+            if events is not None:
+                events[0].append(_event())
+            lla.decode_attn(st["cfg"], L["packed"], st["rope"], t, L["ctx_len"], L["q"],
+                            L["k_self"], L["v_self"], L["positions"], L["q_pos"], L["c_k"],
+                            L["c_v"], out=st["out"], ws=st["ws"])
+            if events is not None:
+                events[1].append(_event())
+    for L in st["layers"]:
+        lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
+
+
+def _event():
+    import torch
+
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def barrier_sync(dist_on):
+    import torch
+    import torch.distributed as dist
+
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_baseline_sample(w, seconds: float, loops=None):
+    """Time the float64 oracle on (b, h) pairs of the workload at full context."""
+    import torch
+    import oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    cfg = O.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
+    cod = synth.workload_codec(w)
+    codec = O.Codec(*(cod[k].astype(np.float64) for k in
+                      ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
+    x = synth.workload_tensors(w, "cpu", seed_offset=99, B=1)
+    arr = {k: (v.float().numpy().astype(np.float64) if v.dtype in (torch.bfloat16, torch.float32)
+               else v.numpy()) for k, v in x.items()}
+    loops = loops or w.loops
+    pairs = 0
+    t0 = time.perf_counter()
+    while True:
+        h = pairs % w.H
+        t = loops[pairs % len(loops)]
+        O.decode_attn_cache(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"], arr["c_k"],
+                            arr["c_v"], arr["positions"], arr["q_pos"], arr["ctx_len"],
+                            pairs=[(0, h)])
+        pairs += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and pairs >= 2:
+            break
+    per_pair = decode_bytes(w, w.n) / (w.B * w.H)
+    return {"value": pairs * per_pair / el / 1e9, "unit": "GB/s", "cores": int(threads),
+            "kind": "oracle", "seconds": round(el, 2),
+            "sample": f"{pairs} (b,h) pairs x {w.n} context tokens, loops {list(loops)}, "
+                      f"float64 NumPy; bytes scaled as the GPU path's algorithmic bytes per pair"}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import looped_transformer_decode_b200 as lla
+
+    w = synth.WORKLOADS[args.workload]
+    st = build_state(w, device)
+    for _ in range(max(args.warmup, 3)):
+        run_step(lla, w, st)
+    barrier_sync(dist_on)
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    ev_pairs = ([], [])
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier_sync(dist_on)
+    start.record()
+    for _ in range(args.steps):
+        run_step(lla, w, st, ev_pairs)
+    stop.record()
+    barrier_sync(dist_on)
+    ms = start.elapsed_time(stop)
+    clk = clocks.stop() if clocks else None
+    dec_ms = [a.elapsed_time(b) for a, b in zip(*ev_pairs)]
+    status = lla.decode_status(st["ws"])
+    if status:
+        raise RuntimeError(f"decode reported device status bits {status}")
+    if dist_on:
+        tt = torch.tensor([ms, float(np.mean(dec_ms))], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, dec_avg = float(tt[0]), float(tt[1])
+    else:
+        dec_avg = float(np.mean(dec_ms))
+
+    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, w.n)
+                      + w.layers * encode_bytes(w, w.encode_tokens))
+    ms_step = ms / args.steps
+    value = world * per_step_bytes / (ms_step * 1e-3) / 1e9
+    ctx_tokens = world * len(w.loops) * w.layers * w.B * w.n / (ms_step * 1e-3)
+    peak, peak_kind = peaks()
+    achieved = decode_bytes(w, w.n) / (dec_avg * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(lla, w, st, args, dist_on, world)
+
+    launches_per_step = (len(w.loops) * w.layers * lla.decode_launches(st["cfg"], w.B, st["n_cap"])
+                         + w.layers)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; latents drawn in latent space as rank-R plus noise)",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "d_head": w.d, "r_k": w.r_k,
+                   "r_v": w.r_v, "mode": "per_head" if w.mode == synth.MODE_PER_HEAD else "lla_2d",
+                   "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
+                   "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2 ({decode_bytes(w, w.n) * w.layers / 1e6:.0f} MB "
+                         "of latents per loop pass)"},
+        "ctx_tokens_per_s": round(ctx_tokens, 1),
+        "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
+        "roofline": {"bound": "hbm", "kernel": "lla_decode_attn (partial + combine)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "decode_call_us": round(dec_avg * 1e3, 2),
+                     "algorithmic_bytes_per_call": decode_bytes(w, w.n)},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(lla, w, st, args, dist_on, world):
+    """Same step with inputs copied from pinned host memory and the output read back."""
+    import torch
+
+    host = []
+    h2d = 0
+    for L in st["layers"]:
+        hl = {k: L[k].cpu().pin_memory() for k in ("c_k", "c_v", "q", "k_self", "v_self",
+                                                    "positions", "q_pos", "ctx_len")}
+        host.append(hl)
+        h2d += sum(v.numel() * v.element_size() for v in hl.values())
+    hx = {"xk": st["xk"].cpu().pin_memory(), "xv": st["xv"].cpu().pin_memory()}
+    h2d += sum(v.numel() * v.element_size() for v in hx.values())
+    out_host = torch.empty(st["out"].shape, dtype=torch.float32).pin_memory()
+    d2h = out_host.numel() * 4 * len(w.loops) * w.layers
+
+    def step():
+        for L, hl in zip(st["layers"], host):
+            for k, v in hl.items():
+                L[k].copy_(v, non_blocking=True)
+        st["xk"].copy_(hx["xk"], non_blocking=True)
+        st["xv"].copy_(hx["xv"], non_blocking=True)
+        for t in w.loops:
+            for L in st["layers"]:
+                lla.decode_attn(st["cfg"], L["packed"], st["rope"], t, L["ctx_len"], L["q"],
+                                L["k_self"], L["v_self"], L["positions"], L["q_pos"], L["c_k"],
+                                L["c_v"], out=st["out"], ws=st["ws"])
+                out_host.copy_(st["out"], non_blocking=True)
+        for L in st["layers"]:
+            lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(2):
+        step()
+    steps = max(3, min(args.steps, 10))
+    barrier_sync(dist_on)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    barrier_sync(dist_on)
+    ms = s.elapsed_time(e) / steps
+    if dist_on:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=st["out"].device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt[0])
+    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, w.n)
+                      + w.layers * encode_bytes(w, w.encode_tokens))
+    return {"value": round(world * per_step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    per_step = max(1.0, args.cpu_seconds / 4)
+    vals = []
+    for _ in range(args.warmup):
+        cpu_baseline_sample(w, per_step / 4)
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline_sample(w, per_step)
+        vals.append(last["value"])
+    el = time.perf_counter() - t0
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "d_head": w.d, "r_k": w.r_k,
+                   "r_v": w.r_v, "batch": w.B, "context": w.n, "layers": w.layers,
+                   "loops": list(w.loops), "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"kind": "oracle", "cores": last["cores"], "value": round(value, 4),
+                         "unit": "GB/s", "sample": last["sample"] + f"; {per_step:.1f} s per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,224 @@
+/*
+ * lla.h -- C ABI of the Looped Latent Attention (LLA) decode library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * What the method computes (pages cited by title and section):
+ *   "Looped Latent Attention: Cross-Loop KV Compression for Looped Transformers"
+ *   (gist.science explainer), Technisches Resümee / Kernmechanismus:
+ *     encode                c    = (x - mu) W_down
+ *     loop-specific decode  x^_t = c W_up,t^T + mu_t
+ *   where x = [x_1; ...; x_T] is one token's pre-RoPE K (or V) for every loop.
+ *   "Looped Latent Attention: 跨循环 KV 压缩精读" (cc.laoqi.cc close reading),
+ *   §二.1 symbol table (W_down is (T d_head) x r, W_up,t is d_head x r),
+ *   §二.2 eq. (4) (exact ratio 2 T d_head / (r_k + r_v)), §二.3 (compress before
+ *   RoPE, rotate the rebuilt K at its position), §二.6 (LLA-2D folds the heads
+ *   into one latent of input width T H d_head; the latent-store path keeps only
+ *   latents and rebuilds on read).
+ *
+ * Conventions
+ *   - Loops are 0-based (t = 0 .. T-1); the pages count from 1.
+ *   - Row vectors, as on the pages.  Every matrix is row-major, C order.
+ *   - bf16 values are passed as their uint16_t bit patterns.
+ *   - RoPE is the split-half layout: pair (i, i + d/2) rotates by angle
+ *     pos * rope_base^(-2 i / d).  Scores are scaled by sm_scale (1/sqrt(d) when 0).
+ *   - The in-flight token (the one whose loops are still running) is not in the
+ *     latent cache: its loop-t K and V are passed exactly (k_self, v_self) and it
+ *     attends to itself at q_pos.  It is encoded with lla_encode after its last loop.
+ *
+ * Ownership and execution
+ *   - Every buffer is allocated by the caller.  Pointers named d_* or documented
+ *     as "device" must be device memory of the current CUDA device; the library
+ *     never allocates device memory, never synchronises the device, and enqueues
+ *     work only on `stream` (a cudaStream_t passed as void*; NULL = legacy stream).
+ *   - Device pointers must be 16-byte aligned; tensors are dense (no strides).
+ *   - Functions are thread-safe; calls on one stream run in order.
+ *
+ * Errors
+ *   Every int-returning function returns LLA_OK (0) or a negative code.  On error
+ *   nothing was enqueued, and lla_last_error() (thread-local) describes it.
+ *   Errors found on the device (positions outside the RoPE table, ctx_len outside
+ *   [0, n_cap], cache slots outside the cache) never fault: the offending element
+ *   is skipped or clamped and a bit is set in a device status word (see below).
+ */
+#ifndef LLA_H_
+#define LLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LLA_OK 0
+#define LLA_ERR_INVALID (-1)     /* null pointer, bad size, misaligned pointer, t >= T ... */
+#define LLA_ERR_UNSUPPORTED (-2) /* shape outside the supported set (see lla_cfg) */
+#define LLA_ERR_TOO_SMALL (-3)   /* packed / table / workspace buffer too small */
+#define LLA_ERR_CUDA (-4)        /* a CUDA call or kernel launch failed */
+
+#define LLA_MODE_PER_HEAD 0 /* one (c_k, c_v) pair per token, layer and head */
+#define LLA_MODE_2D 1       /* LLA-2D: one (c_k, c_v) pair per token and layer */
+
+/* Device status bits (see lla_decode_attn / lla_encode). */
+#define LLA_STATUS_POSITION_RANGE 1 /* a history position or q_pos outside [0, rope_max_pos) */
+#define LLA_STATUS_CTX_RANGE 2      /* ctx_len[b] outside [0, n_cap] (clamped) */
+#define LLA_STATUS_SLOT_RANGE 4     /* an encode slot outside [0, n_slots) (skipped) */
+
+/*
+ * Codec geometry of one shared layer.
+ * Supported: 1 <= T <= 64; 1 <= H <= 128; d_head in {32, 64, 96, 128};
+ * r_k, r_v multiples of 8 in [8, 256]; rope_base > 1; sm_scale >= 0.
+ */
+typedef struct lla_cfg {
+  int32_t T;        /* loops */
+  int32_t H;        /* attention heads (K/V heads; MHA) */
+  int32_t d_head;   /* head width d */
+  int32_t r_k;      /* K latent width */
+  int32_t r_v;      /* V latent width */
+  int32_t mode;     /* LLA_MODE_PER_HEAD or LLA_MODE_2D */
+  float rope_base;  /* RoPE base, e.g. 10000 */
+  float sm_scale;   /* softmax scale; 0 selects 1/sqrt(d_head) */
+} lla_cfg;
+
+/* Last error message of the calling thread ("" if none). Never NULL. */
+const char* lla_last_error(void);
+
+/* Library version string. */
+const char* lla_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Bookkeeping (host only, exact integers).                                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Exact compression ratio of the persistent cache as a reduced fraction num/den.
+ * Per head: 2 T d_head / (r_k + r_v)  (close reading §二.2 eq. (4); gist.science
+ * "Zentrale Beiträge").  LLA-2D: 2 T H d_head / (r_k + r_v)  (close reading §二.6).
+ */
+int lla_ratio(const lla_cfg* cfg, int64_t* num, int64_t* den);
+
+/*
+ * Bytes of bf16 latent cache for `tokens` tokens over `layers` layers:
+ * (r_k + r_v) * H * tokens * layers * 2 per head, (r_k + r_v) * tokens * layers * 2
+ * for LLA-2D.  Also the uncompressed loop-indexed cache (2 T H d_head scalars per
+ * token and layer) when teacher != 0.  Fails with LLA_ERR_INVALID on overflow.
+ */
+int lla_cache_bytes(const lla_cfg* cfg, int64_t tokens, int64_t layers, int teacher,
+                    int64_t* bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Codec packing (once per layer).                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Size in bytes of the packed codec buffer for cfg (0 if cfg is unsupported). */
+size_t lla_codec_packed_bytes(const lla_cfg* cfg);
+
+/*
+ * Pack fp32 codec parameters (device pointers) into the library's internal
+ * device layout.  Inputs (row-major fp32):
+ *   per head:  W_down_{k,v} [H][T*d][r],  W_up_{k,v} [H][T][d][r],  mu_{k,v} [H][T*d]
+ *   LLA-2D:    W_down_{k,v} [T*H*d][r],   W_up_{k,v} [T][H][d][r],  mu_{k,v} [T*H*d]
+ *   (concatenation order: loop-major, then head for LLA-2D, then the d entries.)
+ * The packed buffer (`packed`, device, >= lla_codec_packed_bytes(cfg)) holds W_up
+ * and mu in fp32, W_down rounded to bf16 (round to nearest even), and the encode
+ * bias mu W_down computed with that rounded W_down.  Inputs may be freed once the
+ * stream has passed this call.
+ */
+int lla_codec_pack(const lla_cfg* cfg, const float* W_down_k, const float* W_down_v,
+                   const float* W_up_k, const float* W_up_v, const float* mu_k,
+                   const float* mu_v, void* packed, size_t packed_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* RoPE table (once per d_head / base / maximum position).                    */
+/* ------------------------------------------------------------------------ */
+
+/* Size in bytes of the RoPE table covering positions [0, max_pos). */
+size_t lla_rope_table_bytes(const lla_cfg* cfg, int32_t max_pos);
+
+/*
+ * Fill `table` (device) with (cos, sin) of pos * rope_base^(-2i/d_head) for
+ * pos < max_pos, i < d_head/2, as fp32 pairs [max_pos][d_head/2][2].  Angles are
+ * formed and reduced in fp64 and rounded once to fp32, so large positions keep
+ * full fp32 accuracy (close reading §二.3: full-dimension RoPE on the rebuilt K).
+ */
+int lla_rope_table(const lla_cfg* cfg, int32_t max_pos, void* table, size_t table_bytes,
+                   void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Encode: codec write of finished tokens.                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * c = (x - mu) W_down, rounded to bf16, for n_tok finished tokens
+ * (gist.science, Kernmechanismus, latent storage; close reading §二.6 for LLA-2D).
+ *   x_k, x_v  device bf16 [n_tok][T][H][d]: each token's pre-RoPE K / V rows for all
+ *             loops (the concatenation x = [x_0; ...; x_{T-1}] per head, or over
+ *             (t, h) for LLA-2D).
+ *   slot      device int64 [n_tok]: destination row of each token in the cache.
+ *   c_k, c_v  device bf16 caches with n_slots rows: per head [n_slots][H][r_k] and
+ *             [n_slots][H][r_v]; LLA-2D [n_slots][r_k] and [n_slots][r_v].  A
+ *             cache laid out [B][n_cap][...] is addressed by slot = b * n_cap + j.
+ *   status    optional device int32 (may be NULL): LLA_STATUS_SLOT_RANGE is OR-ed
+ *             in when a slot is outside [0, n_slots); that token is skipped.
+ * n_tok == 0 is a no-op.
+ */
+int lla_encode(const lla_cfg* cfg, const void* packed, int64_t n_tok, const uint16_t* x_k,
+               const uint16_t* x_v, const int64_t* slot, int64_t n_slots, uint16_t* c_k,
+               uint16_t* c_v, int32_t* status, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention over the latent cache at loop t.                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Workspace bytes needed by lla_decode_attn for (cfg, B, n_cap).  The workspace
+ * must be zero-filled once before its first use; the library keeps it consistent
+ * afterwards.  Its first two int32 words are the device status: word 0 collects
+ * the bits of the call in flight, word 1 holds the final bits of the last
+ * completed call (LLA_STATUS_* values).
+ */
+size_t lla_decode_workspace_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap);
+
+/*
+ * out[b][h] = attention of the loop-t query over the history rebuilt from the
+ * latents plus the in-flight token (gist.science Kernmechanismus, loop-specific
+ * reconstruction; close reading §二.3, RoPE after reconstruction):
+ *   k_j  = RoPE(c_k,j W_up,k,t,h^T + mu_k,t,h, positions[b][j])
+ *   s_j  = sm_scale * RoPE(q, q_pos[b]) . k_j ,  s_self likewise with k_self
+ *   p    = softmax over {s_j : j < ctx_len[b]} and s_self
+ *   out  = W_up,v,t,h (sum_j p_j c_v,j) + (sum_j p_j) mu_v,t,h + p_self v_self
+ * (values are summed in latent space and up-projected once; equal to rebuilding
+ * each V because the weights are linear in the rebuilt values.)
+ *   packed        codec from lla_codec_pack (device)
+ *   rope_table    table from lla_rope_table covering [0, rope_max_pos) (device)
+ *   t             loop index, 0 <= t < T
+ *   B, n_cap      batch and cache capacity per sequence (n_cap >= 0)
+ *   ctx_len       device int32 [B]: history length of each sequence (<= n_cap)
+ *   q, k_self, v_self  device fp32 [B][H][d]: the in-flight token's loop-t query,
+ *                 key and value, pre-RoPE
+ *   positions     device int32 [B][n_cap]: position of each history token
+ *   q_pos         device int32 [B]: position of the in-flight token
+ *   c_k, c_v      device bf16 latent caches: per head [B][n_cap][H][r_k] / [..][r_v];
+ *                 LLA-2D [B][n_cap][r_k] / [B][n_cap][r_v]
+ *   out           device fp32 [B][H][d]
+ *   ws            device workspace of >= lla_decode_workspace_bytes(cfg, B, n_cap)
+ * Work is launched on `stream` only; there is no host synchronisation.
+ */
+int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_table,
+                    int32_t rope_max_pos, int32_t t, int32_t B, int32_t n_cap,
+                    const int32_t* ctx_len, const float* q, const float* k_self,
+                    const float* v_self, const int32_t* positions, const int32_t* q_pos,
+                    const uint16_t* c_k, const uint16_t* c_v, float* out, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * Number of kernel launches one lla_decode_attn call makes for (cfg, B, n_cap)
+ * (for launch accounting by callers); -1 if the shape is unsupported.
+ */
+int lla_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLA_H_ */

@@ -1,0 +1,79 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/lla.h"
+
+namespace lla {
+
+// Status words at the head of the decode workspace: [0] bits of the call in
+// flight, [1] bits of the last completed call.  Partials start at kWsHeader.
+constexpr size_t kWsHeader = 256;
+constexpr int kTile = 128;          // history tokens per tile (one per thread / TMEM lane)
+constexpr int kMaxSplits = 64;      // context splits per (b, h) at most
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Offsets (bytes) of each section of the packed codec buffer.
+//   wup_{k,v}  fp32 [T][H][d][r]      loop-t, head-h up-projection W_up,t,h (d x r)
+//   mu_{k,v}   fp32 [T][H][d]         loop-t, head-h mean slice mu_t,h
+//   wd_{k,v}   bf16 [L][r][W]         W_down^T (rows = latent index), L = H (per head) or 1
+//   bias_{k,v} fp32 [L][r]            mu W_down with the bf16-rounded W_down
+struct PackedLayout {
+  size_t wupk, wupv, muk, muv, wdk, wdv, biask, biasv, total;
+  int L;     // latents per token and layer: H (per head) or 1 (LLA-2D)
+  int W;     // encode input width: T*d (per head) or T*H*d (LLA-2D)
+};
+
+PackedLayout packed_layout(const lla_cfg& c);
+
+// Decode split plan shared by the workspace sizing and the launcher.
+struct SplitPlan {
+  int n_tiles;          // ceil(n_cap / kTile)
+  int splits;           // S
+  int tiles_per_split;  // tiles handled by one CTA
+};
+SplitPlan split_plan(const lla_cfg& c, int B, int n_cap);
+size_t partials_bytes(const lla_cfg& c, int B, int S);
+
+// Kernel launchers (return cudaError_t of the launch).
+cudaError_t launch_rope_table(const lla_cfg& c, int max_pos, float2* table, cudaStream_t s);
+cudaError_t launch_pack(const lla_cfg& c, const PackedLayout& L, const float* wdk,
+                        const float* wdv, const float* wupk, const float* wupv,
+                        const float* muk, const float* muv, char* packed, cudaStream_t s);
+cudaError_t launch_encode(const lla_cfg& c, const PackedLayout& L, const char* packed,
+                          int64_t n_tok, const __nv_bfloat16* xk, const __nv_bfloat16* xv,
+                          const int64_t* slot, int64_t n_slots, __nv_bfloat16* ck,
+                          __nv_bfloat16* cv, int32_t* status, cudaStream_t s);
+
+struct DecodeArgs {
+  int T, H, d, r_k, r_v, mode;
+  float kappa;           // sm_scale * log2(e): scores are kept in base-2 units
+  int t, B, n_cap, rope_max_pos;
+  const float* wupk_t;   // packed W_up,k at loop t: [H][d][r_k]
+  const float* wupv_t;   // [H][d][r_v]
+  const float* muk_t;    // [H][d]
+  const float* muv_t;    // [H][d]
+  const float2* rope;    // [rope_max_pos][d/2]
+  const int32_t* ctx_len;
+  const float* q;
+  const float* k_self;
+  const float* v_self;
+  const int32_t* positions;
+  const int32_t* q_pos;
+  const __nv_bfloat16* ck;
+  const __nv_bfloat16* cv;
+  long long lat_tok_k, lat_tok_v;    // elements between consecutive tokens of one sequence
+  long long lat_head_k, lat_head_v;  // elements between heads (0 for LLA-2D)
+  float* out;
+  int32_t* status;       // ws words [0], [1]
+  float* partials;       // [B][H][S][2 + r_v]
+  int S, tiles_per_split;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
+
+}  // namespace lla

@@ -168,3 +168,68 @@ def latents_lowrank_torch(gen, lead_shape, r, R, sigma, device, dtype):
         c = a @ Z + sigma * torch.randn((e - s, r), generator=gen, device=device)
         flat[s:e] = c.to(dtype)
     return out
+
+
+def workload_codec(w: Workload, seed_offset: int = 0):
+    """fp32 codec arrays for a workload: random orthonormal W_down, W_up,t = its loop rows.
+
+    Returns a dict of float32 numpy arrays in the library's input layouts
+    (per head: W_down [H, T*d, r], W_up [H, T, d, r], mu [H, T*d]; LLA-2D:
+    W_down [T*H*d, r], W_up [T, H, d, r], mu [T*H*d]).
+    """
+    g = rng(w.seed * 7919 + seed_offset)
+    T, H, d = w.T, w.H, w.d
+    out = {}
+    for key, r in (("k", w.r_k), ("v", w.r_v)):
+        if w.mode == MODE_PER_HEAD:
+            Wd = np.stack([random_orthonormal(g, T * d, r) for _ in range(H)])
+            Wu = Wd.reshape(H, T, d, r)
+            mu = 0.1 * g.standard_normal((H, T * d))
+        else:
+            Wd = random_orthonormal(g, T * H * d, r)
+            Wu = Wd.reshape(T, H, d, r)
+            mu = 0.1 * g.standard_normal(T * H * d)
+        out["W_down_" + key] = Wd.astype(np.float32)
+        out["W_up_" + key] = np.ascontiguousarray(Wu).astype(np.float32)
+        out["mu_" + key] = mu.astype(np.float32)
+    return out
+
+
+def workload_tensors(w: Workload, device, seed_offset: int = 0, B: int | None = None,
+                     n: int | None = None):
+    """Device tensors of one decode step of workload ``w`` (one layer).
+
+    Latents are drawn directly in latent space (rank-R plus noise, bf16);
+    positions are 0..n-1 with the in-flight token at n; q ~ N(0,1)/sqrt(d);
+    k_self, v_self ~ N(0, 0.2^2).
+    """
+    import torch
+
+    B = w.B if B is None else B
+    n = w.n if n is None else n
+    tg = torch.Generator(device=device)
+    tg.manual_seed(w.seed * 104729 + seed_offset)
+    lead = (B, n, w.H) if w.mode == MODE_PER_HEAD else (B, n)
+    t = {
+        "c_k": latents_lowrank_torch(tg, lead, w.r_k, w.R, 0.01, device, torch.bfloat16),
+        "c_v": latents_lowrank_torch(tg, lead, w.r_v, w.R, 0.01, device, torch.bfloat16),
+        "positions": torch.arange(n, device=device, dtype=torch.int32).repeat(B, 1).contiguous(),
+        "q_pos": torch.full((B,), n, device=device, dtype=torch.int32),
+        "ctx_len": torch.full((B,), n, device=device, dtype=torch.int32),
+        "q": torch.randn((B, w.H, w.d), generator=tg, device=device) / float(np.sqrt(w.d)),
+        "k_self": 0.2 * torch.randn((B, w.H, w.d), generator=tg, device=device),
+        "v_self": 0.2 * torch.randn((B, w.H, w.d), generator=tg, device=device),
+    }
+    return t
+
+
+def encode_inputs(w: Workload, device, n_tok: int, seed_offset: int = 0):
+    """bf16 per-loop K/V rows [n_tok, T, H, d] for encode, trajectory-shaped magnitudes."""
+    import torch
+
+    tg = torch.Generator(device=device)
+    tg.manual_seed(w.seed * 15485863 + seed_offset)
+    shape = (n_tok, w.T, w.H, w.d)
+    xk = (0.3 * torch.randn(shape, generator=tg, device=device)).to(torch.bfloat16)
+    xv = (0.3 * torch.randn(shape, generator=tg, device=device)).to(torch.bfloat16)
+    return xk, xv

@@ -1,0 +1,199 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Tolerances (written here, from the contract): attention outputs within 2e-3 max
+relative error per (b, h); encoded latents within 1e-2 of the latent's L2 norm
+(against the unrounded fp64 value); RoPE table within 1e-7 absolute; status
+bits and bookkeeping exact.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import synth
+from cases import ATTN_TOL, LATENT_TOL, decode_case, expected, f32, rel_err
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import looped_transformer_decode_b200 as lla
+    from gpu_util import DeviceCase, bf16_tensor, f32_tensor, i32_tensor, lib_cfg, pack
+
+
+# ----------------------------------------------------------------------------- RoPE table
+
+@pytest.mark.parametrize("d", [32, 96, 128])
+def test_rope_table_matches_fp64_angles(d):
+    cfg = lla.Cfg(1, 1, d, 8, 8, rope_base=10000.0)
+    max_pos = 40000
+    tab = lla.rope_table(cfg, max_pos).cpu().numpy().astype(np.float64)
+    ang = np.arange(max_pos)[:, None] * O.rope_inv_freq(d, 10000.0)[None]
+    np.testing.assert_allclose(tab[..., 0], np.cos(ang), atol=1e-7, rtol=0)
+    np.testing.assert_allclose(tab[..., 1], np.sin(ang), atol=1e-7, rtol=0)
+
+
+# ----------------------------------------------------------------------------- encode
+
+ENCODE_CFGS = [
+    O.Cfg(4, 2, 64, 8, 16),                       # tiny per-head workload
+    O.Cfg(4, 16, 128, 96, 160),                   # per-head 4x
+    O.Cfg(4, 16, 128, 16, 32),                    # per-head 21.3x
+    O.Cfg(32, 2, 96, 64, 128),                    # deep loop, two heads
+    O.Cfg(2, 4, 64, 32, 48, O.MODE_2D),           # LLA-2D small
+    O.Cfg(4, 16, 128, 64, 128, O.MODE_2D),        # LLA-2D workload width
+]
+
+
+@pytest.mark.parametrize("cfg", ENCODE_CFGS, ids=lambda c: f"T{c.T}H{c.H}d{c.d}r{c.r_k}_{c.r_v}m{c.mode}")
+def test_encode_matches_oracle(cfg):
+    case = decode_case(cfg, 1, 4, seed=50 + cfg.r_k, R=3)
+    g = synth.rng(77)
+    shared = cfg.mode == O.MODE_2D
+    mk = synth.trajectory_model(g, cfg.T, cfg.H, cfg.d, 3, shared=shared)
+    n_tok, n_slots = 37, 50
+    xk = O.bf16_round(synth.sample_trajectories(g, mk, n_tok))
+    xv = O.bf16_round(synth.sample_trajectories(g, mk, n_tok))
+    slot = g.permutation(n_slots)[:n_tok]
+    packed = pack(case)
+    L = cfg.H if cfg.mode == O.MODE_PER_HEAD else 1
+    lead = (n_slots, cfg.H) if cfg.mode == O.MODE_PER_HEAD else (n_slots,)
+    ck = torch.zeros((*lead, cfg.r_k), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros((*lead, cfg.r_v), dtype=torch.bfloat16, device="cuda")
+    lla.encode(lib_cfg(cfg), packed, bf16_tensor(xk), bf16_tensor(xv),
+               torch.from_numpy(slot.astype(np.int64)).cuda(), ck, cv)
+    torch.cuda.synchronize()
+    want_k, want_v = O.encode_tokens(cfg, case.codec, xk, xv)
+    got_k = ck.float().cpu().numpy().astype(np.float64)[slot]
+    got_v = cv.float().cpu().numpy().astype(np.float64)[slot]
+    for got, want in ((got_k, want_k), (got_v, want_v)):
+        got = got.reshape(n_tok, L, -1)
+        want = want.reshape(n_tok, L, -1)
+        err = np.abs(got - want).max(-1) / np.linalg.norm(want, axis=-1)
+        assert err.max() <= LATENT_TOL, err.max()
+    # rows that received no token stay untouched
+    untouched = np.setdiff1d(np.arange(n_slots), slot)
+    assert np.all(ck.float().cpu().numpy()[untouched] == 0)
+
+
+def test_encode_out_of_range_slot_sets_status_and_skips():
+    cfg = O.Cfg(4, 2, 64, 8, 16)
+    case = decode_case(cfg, 1, 4, seed=3)
+    packed = pack(case)
+    x = bf16_tensor(O.bf16_round(0.3 * synth.rng(1).standard_normal((3, 4, 2, 64))))
+    ck = torch.zeros((5, 2, 8), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros((5, 2, 16), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    slot = torch.tensor([0, 5, -1], dtype=torch.int64, device="cuda")
+    lla.encode(lib_cfg(cfg), packed, x, x, slot, ck, cv, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == lla.STATUS_SLOT_RANGE
+    assert ck[0].abs().sum() > 0 and ck[1:].abs().sum() == 0
+
+
+# ----------------------------------------------------------------------------- decode, small
+
+SMALL = [
+    # (cfg, B, n_cap, ctx_len, kwargs)
+    (O.Cfg(4, 2, 64, 8, 16), 1, 128, None, {}),                                  # tiny workload
+    (O.Cfg(4, 3, 64, 16, 24), 3, 300, [300, 129, 1], {}),                        # ragged tails
+    (O.Cfg(4, 2, 128, 96, 160), 2, 520, [520, 385], {}),
+    (O.Cfg(4, 2, 96, 64, 128), 2, 700, [700, 256], {"R": 8, "gamma": 0.85}),
+    (O.Cfg(3, 2, 32, 8, 8), 2, 130, [130, 0], {}),                               # empty history
+    (O.Cfg(4, 2, 64, 16, 32), 1, 2000, None, {}),                                # many splits
+    (O.Cfg(4, 2, 64, 24, 40), 2, 200, None, {"codec": "random"}),                # no SVD structure
+    (O.Cfg(4, 2, 64, 16, 32), 2, 200, None, {"q_scale": 25.0}),                  # sharp softmax
+    (O.Cfg(4, 2, 64, 16, 32), 2, 260, None, {"positions": "random"}),            # arbitrary positions
+    (O.Cfg(2, 4, 64, 32, 48, O.MODE_2D), 2, 200, [200, 77], {}),                 # LLA-2D
+    (O.Cfg(4, 4, 128, 64, 128, O.MODE_2D), 1, 300, None, {"q_scale": 10.0}),
+]
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: f"T{s[0].T}H{s[0].H}d{s[0].d}r{s[0].r_k}_{s[0].r_v}m{s[0].mode}B{s[1]}n{s[2]}")
+def test_decode_matches_oracle_small(spec):
+    cfg, B, n_cap, ctx, kw = spec
+    case = decode_case(cfg, B, n_cap, seed=100 + n_cap, ctx_len=ctx, **kw)
+    dev = DeviceCase(case)
+    for t in range(cfg.T):
+        got = dev.decode(t)
+        want = expected(case, t)
+        err = rel_err(got, want)
+        assert np.isfinite(got).all()
+        assert err.max() <= ATTN_TOL, (t, err.max())
+    assert lla.decode_status(dev.ws) == 0
+
+
+def test_decode_status_bits_for_bad_device_inputs():
+    cfg = O.Cfg(4, 2, 64, 16, 32)
+    case = decode_case(cfg, 2, 200, seed=9)
+    dev = DeviceCase(case, rope_max_pos=201)
+    dev.decode(0)
+    assert lla.decode_status(dev.ws) == 0
+    bad = case.positions.copy()
+    bad[0, 10] = 5000                         # outside the RoPE table
+    dev.positions = i32_tensor(bad)
+    out = dev.decode(0)
+    assert np.isfinite(out).all()
+    assert lla.decode_status(dev.ws) & lla.STATUS_POSITION_RANGE
+    dev.positions = i32_tensor(case.positions)
+    dev.ctx_len = i32_tensor([250, 200])      # above n_cap: clamped
+    out = dev.decode(0)
+    assert np.isfinite(out).all()
+    assert lla.decode_status(dev.ws) == lla.STATUS_CTX_RANGE
+    dev.ctx_len = i32_tensor(case.ctx_len)
+    dev.decode(0)
+    assert lla.decode_status(dev.ws) == 0
+
+
+def test_decode_is_deterministic():
+    cfg = O.Cfg(4, 2, 128, 96, 160)
+    case = decode_case(cfg, 2, 700, seed=12)
+    dev = DeviceCase(case)
+    a, b = dev.decode(2), dev.decode(2)
+    np.testing.assert_array_equal(a, b)
+
+
+# ----------------------------------------------------------------------------- decode, full size
+
+def _sample_pairs(B, H, k, seed):
+    g = synth.rng(seed)
+    pairs = {(B - 1, H - 1), (0, 0)}
+    while len(pairs) < min(k, B * H):
+        pairs.add((int(g.integers(B)), int(g.integers(H))))
+    return sorted(pairs)
+
+
+@pytest.mark.parametrize("name", synth.WORKLOAD_ORDER[1:])
+def test_decode_full_size_sampled(name):
+    """Full-size workloads in the bench's launch configuration, sampled (b, h) pairs."""
+    w = synth.WORKLOADS[name]
+    cfg = O.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
+    lc = lib_cfg(cfg)
+    codec_np = synth.workload_codec(w)
+    codec = O.Codec(*(codec_np[k].astype(np.float64) for k in
+                      ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
+    packed = lla.codec_pack(lc, *(torch.from_numpy(codec_np[k]).cuda() for k in
+                                  ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
+    x = synth.workload_tensors(w, "cuda")
+    rope = lla.rope_table(lc, w.n + 1)
+    ws = lla.decode_workspace(lc, w.B, w.n)
+    pairs = _sample_pairs(w.B, w.H, 48, w.seed)
+    bs = sorted({b for b, _ in pairs})
+    ck = x["c_k"][bs].float().cpu().numpy().astype(np.float64)
+    cv = x["c_v"][bs].float().cpu().numpy().astype(np.float64)
+    remap = {b: i for i, b in enumerate(bs)}
+    for t in w.loops:
+        out = lla.decode_attn(lc, packed, rope, t, x["ctx_len"], x["q"], x["k_self"], x["v_self"],
+                              x["positions"], x["q_pos"], x["c_k"], x["c_v"], ws=ws)
+        torch.cuda.synchronize()
+        got = out.double().cpu().numpy()
+        sub = [(remap[b], h) for b, h in pairs]
+        sel = lambda a: a[bs]  # noqa: E731
+        want = O.decode_attn_cache(cfg, codec, t, sel(x["q"].double().cpu().numpy()),
+                                   sel(x["k_self"].double().cpu().numpy()),
+                                   sel(x["v_self"].double().cpu().numpy()), ck, cv,
+                                   sel(x["positions"].cpu().numpy()), sel(x["q_pos"].cpu().numpy()),
+                                   sel(x["ctx_len"].cpu().numpy()), pairs=sub)
+        for (b, h), (i, _) in zip(pairs, sub):
+            e = np.abs(got[b, h] - want[i, h]).max() / np.abs(want[i, h]).max()
+            assert e <= ATTN_TOL, (name, t, b, h, e)
+    assert lla.decode_status(ws) == 0
