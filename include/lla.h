@@ -212,6 +212,38 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
                     size_t ws_bytes, void* stream);
 
 /*
+ * lla_decode_attn for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this entry point; it exists for deployment.
+ * Some callers cannot call cudaMalloc or any other allocator when they run
+ * decode: code inside an allocator-free region of a host runtime, plugins that
+ * are handed only their input and output buffers, or servers that forbid
+ * allocation after start-up so that their memory use stays fixed.  This call
+ * computes exactly what lla_decode_attn computes (same kernels, same arguments
+ * and layouts) but takes no workspace: its split partials and status words live
+ * in a fixed device array of 8 MiB (8388608 bytes) that the library holds on
+ * every GPU where it is loaded, until the process exits.
+ *   - Shapes whose workspace (lla_decode_workspace_bytes) exceeds 8 MiB are
+ *     rejected with LLA_ERR_TOO_SMALL before anything is enqueued.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.  Later calls reuse the address.
+ *   - All calls share the one array and it keeps the last call's contents.  Each
+ *     call clears the status words it needs; calls that overlap on the GPU (on
+ *     different streams, or from different threads) race on the array and must
+ *     be serialised by the caller.
+ *   - status_out: optional device int32 (may be NULL) that receives this call's
+ *     LLA_STATUS_* bits, written on `stream` after the kernels.
+ * It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+int lla_decode_attn_noalloc(const lla_cfg* cfg, const void* packed, const void* rope_table,
+                            int32_t rope_max_pos, int32_t t, int32_t B, int32_t n_cap,
+                            const int32_t* ctx_len, const float* q, const float* k_self,
+                            const float* v_self, const int32_t* positions,
+                            const int32_t* q_pos, const uint16_t* c_k, const uint16_t* c_v,
+                            float* out, int32_t* status_out, void* stream);
+
+/*
  * Number of kernel launches one lla_decode_attn call makes for (cfg, B, n_cap)
  * (for launch accounting by callers); -1 if the shape is unsupported.
  */

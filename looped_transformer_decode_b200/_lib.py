@@ -75,6 +75,8 @@ SIGNATURES = {
     "lla_decode_attn": (ctypes.c_int, [_CFG, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P,
                                        _P, _P, _P, _P, _P, _SZ, _P]),
     "lla_decode_launches": (ctypes.c_int, [_CFG, _I32, _I32]),
+    "lla_decode_attn_noalloc": (ctypes.c_int, [_CFG, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P,
+                                               _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(lib, _name)

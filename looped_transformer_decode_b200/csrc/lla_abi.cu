@@ -120,6 +120,16 @@ size_t partials_bytes(const lla_cfg& c, int B, int S) {
   return (size_t)B * c.H * S * (2 + c.r_v) * sizeof(float);
 }
 
+int set_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
 }  // namespace lla
 
 using namespace lla;

@@ -76,4 +76,7 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
 
+// Record `fmt` as the calling thread's lla_last_error() message; returns `code`.
+int set_error(int code, const char* fmt, ...);
+
 }  // namespace lla

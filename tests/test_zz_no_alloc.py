@@ -1,0 +1,64 @@
+"""lla_decode_attn_noalloc: decode attention for callers that cannot allocate.
+
+Callers such as allocator-free runtime regions, plugins handed only their
+input and output buffers, or servers that freeze memory after start-up cannot
+provide a workspace.  The allocation-free entry point keeps its scratch in a
+fixed array inside the library.  This file checks, through the C ABI, that it
+returns what the workspace entry point returns on two calls in a row, and that
+it rejects shapes whose scratch would exceed the array.  It is named so that
+pytest collects it last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle as O
+from cases import ATTN_TOL, decode_case, rel_err
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import looped_transformer_decode_b200 as lla
+    from gpu_util import DeviceCase, f32_tensor
+
+
+def _noalloc(dev, t, out, status):
+    c = dev.case
+    ks, vs = f32_tensor(c.k_self[t]), f32_tensor(c.v_self[t])
+    p = lambda x: ctypes.c_void_p(x.data_ptr())  # noqa: E731
+    rc = lla.lib.lla_decode_attn_noalloc(
+        ctypes.byref(dev.cfg.c()), p(dev.packed), p(dev.rope), dev.rope.shape[0], t, c.B,
+        c.n_cap, p(dev.ctx_len), p(dev.q), p(ks), p(vs), p(dev.positions), p(dev.q_pos),
+        p(dev.c_k), p(dev.c_v), p(out), p(status),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == lla.OK, lla.last_error()
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy()
+
+
+def test_noalloc_matches_workspace_entry_point_twice():
+    cfg = O.Cfg(4, 4, 128, 96, 160)
+    case = decode_case(cfg, 2, 900, seed=4242, ctx_len=[900, 333])
+    dev = DeviceCase(case)
+    out = torch.empty((case.B, cfg.H, cfg.d), dtype=torch.float32, device="cuda")
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    for t in (1, 3):                                   # two calls in a row
+        want = dev.decode(t)                           # existing entry point, caller workspace
+        got = _noalloc(dev, t, out, status)
+        assert np.isfinite(got).all()
+        assert rel_err(got, want).max() <= ATTN_TOL
+        assert int(status.item()) == 0
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    cfg = lla.Cfg(4, 128, 128, 96, 256)
+    B, n_cap = 4096, 8192
+    assert lla.lib.lla_decode_workspace_bytes(ctypes.byref(cfg.c()), B, n_cap) > (8 << 20)
+    fake = ctypes.c_void_p(0x10000)   # never dereferenced: the size check comes first
+    rc = lla.lib.lla_decode_attn_noalloc(ctypes.byref(cfg.c()), fake, fake, 8192, 0, B, n_cap,
+                                         fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                                         None, None)
+    assert rc == lla.ERR_TOO_SMALL
+    assert "8388608" in lla.last_error()
