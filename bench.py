@@ -36,8 +36,8 @@ METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop st
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="lla", choices=["lla", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -85,7 +85,7 @@ class ClockSampler:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-i", str(gpu_index), "-lms", "200"], stdout=self.f,
+                                       "-i", str(gpu_index), "-lms", "20"], stdout=self.f,
                                       stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.p = None

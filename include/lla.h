@@ -63,6 +63,7 @@ extern "C" {
 #define LLA_STATUS_POSITION_RANGE 1 /* a history position or q_pos outside [0, rope_max_pos) */
 #define LLA_STATUS_CTX_RANGE 2      /* ctx_len[b] outside [0, n_cap] (clamped) */
 #define LLA_STATUS_SLOT_RANGE 4     /* an encode slot outside [0, n_slots) (skipped) */
+#define LLA_STATUS_TIMEOUT 8        /* a kernel wait timed out; that call's output is invalid */
 
 /*
  * Codec geometry of one shared layer.

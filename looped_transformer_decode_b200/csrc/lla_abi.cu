@@ -105,6 +105,13 @@ SplitPlan split_plan(const lla_cfg& c, int B, int n_cap) {
     p.tiles_per_split = 0;
     return p;
   }
+  int S_tc = 0, tps_tc = 0;
+  if (decode_tc_plan(c, B, n_cap, &S_tc, &tps_tc)) {
+    p.splits = S_tc;
+    p.tiles_per_split = tps_tc;
+    p.tensor_cores = true;
+    return p;
+  }
   // Aim for about four resident CTAs per SM on a 148-SM part.
   const long long units = (long long)B * c.H;
   long long want = (4 * 148 + units - 1) / units;
@@ -332,7 +339,12 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   a.S = plan.splits;
   a.tiles_per_split = plan.tiles_per_split;
   int launches = 0;
-  cudaError_t ce = launch_decode(a, static_cast<cudaStream_t>(stream), &launches);
+  cudaError_t ce = cudaErrorNotSupported;
+  if (plan.tensor_cores && plan.splits > 0) {
+    ce = launch_decode_tc(*cfg, a, static_cast<cudaStream_t>(stream));
+    if (ce == cudaSuccess) ce = launch_combine(a, static_cast<cudaStream_t>(stream));
+  }
+  if (ce == cudaErrorNotSupported) ce = launch_decode(a, static_cast<cudaStream_t>(stream), &launches);
   if (ce != cudaSuccess) return cuda_fail(ce, "lla_decode_attn launch");
   return ok();
 }

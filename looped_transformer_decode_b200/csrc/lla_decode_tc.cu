@@ -1,0 +1,729 @@
+// Per-head LLA decode attention on the 5th-generation tensor cores (sm_100a).
+//
+// Same arithmetic as the CUDA-core kernel (query folded into the K
+// up-projection, RoPE as a complex product with the fp64-built table, base-2
+// online softmax, V summed in latent space), reorganised for B200:
+//
+//   * persistent CTAs, one per SM, walk a list of work items (sequence b, group
+//     of G heads, context split s); the split partials feed the combine pass;
+//   * warp 0 streams 128-token tiles of c_k and c_v with TMA into an NST-deep
+//     shared-memory ring (c_k tiles land in the swizzled K-major layout the
+//     tensor core reads);
+//   * warp 1 issues tcgen05.mma: U[128 x d] = C_k[128 x r_k] * A~^T[r_k x d] per
+//     head, plus one K=16 MMA with a ones column that adds the per-column bias
+//     M~ (split into bf16 hi + lo), accumulating in fp32 in TMEM;
+//   * warps 2..9 (two warpgroups, each owning half of the RoPE pairs of every
+//     token row) read U from TMEM, form s_j = sum_i Re(U_ji e^{i p_j theta_i}),
+//     run the online softmax, and accumulate sum_j p_j c_v,j from the staged c_v
+//     tile; between items they rebuild A~ and M~ for the next (b, heads) in
+//     shared memory.
+// The close reading §二.3 fixes the order (rebuild K, then RoPE at its
+// position); folding q into W_up and RoPE into a complex dot product changes
+// only the order of the same sums.
+//
+// Every wait is bounded (lla_sm100.cuh); on a timeout the CTA records
+// LLA_STATUS_TIMEOUT, drains its in-flight copies, frees TMEM and returns.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "lla_internal.cuh"
+#include "lla_sm100.cuh"
+
+namespace lla {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;       // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kSmemLimit = 232448;  // per-block dynamic shared memory on sm_100
+
+struct TcParams {
+  int H, r_k, r_v, K_pad, box_k, nkb, swz;   // swz: descriptor swizzle code
+  int Q, nv_items;                           // V-phase split: token residues, work items
+  int B, n_cap, S, tps, HG, n_items, rope_max_pos;
+  float kappa;
+  uint32_t st_off, st_bytes, cv_off, box_bytes;
+  uint32_t b_off, b_head_bytes, b_sbo, ones_off, bias_off, qc_off, sbuf_off, p_off, red_off,
+      alpha_off, obuf_off, bar_off, misc_off;
+  int nst, nacc, acc_cols, tmem_cols;
+  uint32_t tx_bytes;
+  const float* wupk_t;   // [H][d][r_k]
+  const float* muk_t;    // [H][d]
+  const float2* rope;    // [rope_max_pos][d/2]
+  const int32_t* ctx_len;
+  const float* q;        // [B][H][d]
+  const int32_t* positions;
+  const int32_t* q_pos;
+  int32_t* status;
+  float* partials;       // [B][H][S][2 + r_v]
+};
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// bar.red.or over the 256 epilogue threads (named barrier 1): returns the OR of `pred`.
+__device__ __forceinline__ int epi_barrier_or(int pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.red.or.pred po, 1, 256, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred)
+      : "memory");
+  return static_cast<int>(out);
+}
+
+struct ItemRange {
+  int b, hg, s, tok0, tok_end, ntiles;
+};
+
+__device__ __forceinline__ ItemRange item_range(const TcParams& p, int item, bool flag_ctx) {
+  ItemRange r;
+  r.s = item % p.S;
+  const int u = item / p.S;
+  r.hg = u % p.HG;
+  r.b = u / p.HG;
+  int n = p.ctx_len[r.b];
+  if (n < 0 || n > p.n_cap) {
+    if (flag_ctx) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
+    n = n < 0 ? 0 : p.n_cap;
+  }
+  r.tok0 = r.s * p.tps * kTile;
+  r.tok_end = min(r.tok0 + p.tps * kTile, n);
+  r.ntiles = r.tok_end > r.tok0 ? (r.tok_end - r.tok0 + kTile - 1) / kTile : 0;
+  return r;
+}
+
+// Rebuild the MMA B operand A~ (no-swizzle K-major, rows n = 2i (Re) / 2i+1 (Im))
+// and the bias tile for item (b, head group) in shared memory.  All 256 epilogue
+// threads take part; ends with the proxy fence and an epilogue barrier.
+template <int D, int G>
+__device__ void prepare_item(const TcParams& p, unsigned char* sm, int et, int b, int hg) {
+  constexpr int HALF = D / 2;
+  float2* qc = reinterpret_cast<float2*>(sm + p.qc_off);
+  int qp = p.q_pos[b];
+  if (qp < 0 || qp >= p.rope_max_pos) {
+    if (et == 0) atomicOr(p.status, LLA_STATUS_POSITION_RANGE);
+    qp = 0;
+  }
+  for (int idx = et; idx < G * HALF; idx += kEpiThreads) {
+    const int g = idx / HALF, i = idx % HALF;
+    const int h = hg * G + g;
+    const float2 e = p.rope[(size_t)qp * HALF + i];
+    const float* qh = p.q + ((size_t)b * p.H + h) * D;
+    const float x0 = qh[i], x1 = qh[i + HALF];
+    qc[idx] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
+  }
+  named_barrier(1, kEpiThreads);
+  const int Kp = p.K_pad;
+  for (int idx = et; idx < G * D * Kp; idx += kEpiThreads) {
+    const int k = idx % Kp;
+    const int n = (idx / Kp) % D;
+    const int g = idx / (D * Kp);
+    const int h = hg * G + g;
+    const int i = n >> 1;
+    float val = 0.f;
+    if (k < p.r_k) {
+      const float* W = p.wupk_t + (size_t)h * D * p.r_k;
+      const float wr = W[(size_t)i * p.r_k + k], wi = W[(size_t)(i + HALF) * p.r_k + k];
+      const float2 z = qc[g * HALF + i];
+      val = (n & 1) ? p.kappa * (z.x * wi - z.y * wr) : p.kappa * (z.x * wr + z.y * wi);
+    }
+    const uint32_t off = p.b_off + g * p.b_head_bytes + (n >> 3) * p.b_sbo + (k >> 3) * 128 +
+                         (n & 7) * 16 + (k & 7) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(sm + off) = __float2bfloat16_rn(val);
+  }
+  for (int idx = et; idx < G * D; idx += kEpiThreads) {
+    const int n = idx % D, g = idx / D;
+    const int h = hg * G + g;
+    const int i = n >> 1;
+    const float* mu = p.muk_t + (size_t)h * D;
+    const float mr = mu[i], mi = mu[i + HALF];
+    const float2 z = qc[g * HALF + i];
+    const float val = (n & 1) ? p.kappa * (z.x * mi - z.y * mr) : p.kappa * (z.x * mr + z.y * mi);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(val);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
+    const uint32_t off = p.bias_off + g * (D * 16 * 2) + (n >> 3) * 256 + (n & 7) * 16;
+    *reinterpret_cast<__nv_bfloat16*>(sm + off) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(sm + off + 2) = lo;
+  }
+  fence_proxy_async_smem();
+  named_barrier(1, kEpiThreads);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap map_k,
+                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
+  constexpr int HALF = D / 2;
+  constexpr int WG_PAIRS = D / 4;   // RoPE pairs per epilogue warpgroup
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + p.bar_off);
+  uint64_t* empty = full + p.nst;
+  uint64_t* tfull = empty + p.nst;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* bop = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.nst; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 8);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);
+    }
+    mbar_init(bop, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    const int et = threadIdx.x - 64;
+    // ones tile [128 x 16]: columns 0 and 1 hold 1.0; bias tiles start at zero.
+    for (int idx = et; idx < 128 * 16; idx += kEpiThreads) {
+      const int m = idx / 16, k = idx % 16;
+      const uint32_t off = p.ones_off + (m >> 3) * 256 + (k >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2;
+      *reinterpret_cast<__nv_bfloat16*>(sm + off) = __float2bfloat16_rn(k < 2 ? 1.f : 0.f);
+    }
+    for (int idx = et; idx < G * D * 16; idx += kEpiThreads)
+      reinterpret_cast<__nv_bfloat16*>(sm + p.bias_off)[idx] = __float2bfloat16_rn(0.f);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, item, false);
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
+          if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], p.tx_bytes);
+          unsigned char* st = sm + p.st_off + stage * p.st_bytes;
+          const int y = r.tok0 + k * kTile;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const int h = r.hg * G + g;
+            for (int kb = 0; kb < p.nkb; ++kb)
+              tma_load_3d(st + (g * p.nkb + kb) * p.box_bytes, &map_k, &full[stage],
+                          h * p.r_k + kb * p.box_k, y, r.b);
+            tma_load_3d(st + p.cv_off + g * (kTile * p.r_v * 2), &map_v, &full[stage], h * p.r_v,
+                        y, r.b);
+          }
+        }
+      }
+      if (!ok) {
+        // Drain: wait (bounded) for every copy this thread issued before leaving.
+        const uint32_t n_out = it < (uint32_t)p.nst ? it : (uint32_t)p.nst;
+        for (uint32_t j = 0; j < n_out; ++j) {
+          const uint32_t i = it - 1 - j;
+          const uint32_t stage = i % p.nst, ph = (i / p.nst) & 1u;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[stage], ph) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D);
+      const uint32_t sbo_a = 16u * p.box_k;
+      const uint32_t ones_addr = smem_addr(sm + p.ones_off);
+      uint32_t it = 0, item_no = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, item, false);
+        if (r.ntiles == 0) continue;   // no tiles: the epilogue prepares nothing either
+        if (!mbar_wait(bop, item_no & 1u, abort_flag)) break;
+        ++item_no;
+        tc_fence_after();
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
+          const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+          if (!mbar_wait(&full[stage], ph, abort_flag) ||
+              !mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st_addr = smem_addr(sm + p.st_off + stage * p.st_bytes);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint32_t d_tmem = tmem_base + acc * p.acc_cols + g * D;
+            const uint32_t b_addr = smem_addr(sm + p.b_off + g * p.b_head_bytes);
+            for (int kk = 0; kk < p.K_pad / 16; ++kk) {
+              const int kb = (kk * 16) / p.box_k, kin = (kk * 16) % p.box_k;
+              const uint64_t adesc =
+                  smem_desc(st_addr + (g * p.nkb + kb) * p.box_bytes + kin * 2, 16, sbo_a, p.swz);
+              const uint64_t bdesc = smem_desc(b_addr + kk * 256, 128, p.b_sbo, 0);
+              mma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            }
+            const uint64_t odesc = smem_desc(ones_addr, 128, 256, 0);
+            const uint64_t bias_desc =
+                smem_desc(smem_addr(sm + p.bias_off + g * (D * 16 * 2)), 128, 256, 0);
+            mma_bf16(d_tmem, odesc, bias_desc, idesc, 1u);
+          }
+          mma_commit(&tfull[acc]);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;
+    const int wgi = (warp - 2) >> 2;          // which half of the RoPE pairs
+    const int sub = warp & 3;                 // TMEM sub-partition of this warp
+    const int row = sub * 32 + lane;          // token row of the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+    float* sbuf = reinterpret_cast<float*>(sm + p.sbuf_off);   // [G][128]
+    float* P = reinterpret_cast<float*>(sm + p.p_off);         // [G][128]
+    float* red = reinterpret_cast<float*>(sm + p.red_off);     // [G][4]
+    float* alpha_s = reinterpret_cast<float*>(sm + p.alpha_off);
+    float* obuf = reinterpret_cast<float*>(sm + p.obuf_off);   // [Q][G][r_v]
+    const int rv2 = p.r_v >> 1;
+
+    uint32_t it = 0;
+    bool aborted = false;
+    for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
+      const ItemRange r = item_range(p, item, et == 0);
+      if (r.ntiles > 0) {
+        // The previous item's MMAs have all completed (its last tile was read from
+        // TMEM), so the B operand can be rebuilt; one arrival per non-empty item.
+        prepare_item<D, G>(p, sm, et, r.b, r.hg);
+        if (et == 0) mbar_arrive(bop);
+      }
+      float m_run[G], l_part[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        m_run[g] = -INFINITY;
+        l_part[g] = 0.f;
+      }
+      float o[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      for (int k = 0; k < r.ntiles; ++k, ++it) {
+        const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
+        const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+        const int t0 = r.tok0 + k * kTile;
+        const int cnt = min(kTile, r.tok_end - t0);
+        const bool valid = row < cnt;
+        int pos = 0;
+        if (valid) {
+          pos = p.positions[(size_t)r.b * p.n_cap + t0 + row];
+          if (pos < 0 || pos >= p.rope_max_pos) {
+            atomicOr(p.status, LLA_STATUS_POSITION_RANGE);
+            pos = 0;
+          }
+        }
+        float4 e4[WG_PAIRS / 2];
+        const float4* erow =
+            reinterpret_cast<const float4*>(p.rope + (size_t)pos * HALF + wgi * WG_PAIRS);
+#pragma unroll
+        for (int c = 0; c < WG_PAIRS / 2; ++c) e4[c] = erow[c];
+
+        bool ok = mbar_wait(&tfull[acc], aph, abort_flag);
+        tc_fence_after();
+        float part[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          part[g] = 0.f;
+          const uint32_t col = tmem_base + lane_addr + acc * p.acc_cols + g * D + wgi * HALF;
+          float u[HALF];
+#pragma unroll
+          for (int c = 0; c < HALF / 16; ++c) tmem_ld16(col + c * 16, u + c * 16);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q2 = 0; q2 < HALF / 4; ++q2) {
+            const float4 e = e4[q2];   // (cos, sin) of two consecutive pairs
+            part[g] = fmaf(u[4 * q2], e.x, part[g]);
+            part[g] = fmaf(-u[4 * q2 + 1], e.y, part[g]);
+            part[g] = fmaf(u[4 * q2 + 2], e.z, part[g]);
+            part[g] = fmaf(-u[4 * q2 + 3], e.w, part[g]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        ok = ok && mbar_wait(&full[stage], ph, abort_flag);
+        if (wgi == 1) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) sbuf[g * kTile + row] = part[g];
+        }
+        if (epi_barrier_or(!ok)) {
+          aborted = true;
+          break;
+        }
+        if (wgi == 0) {
+          float s[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            s[g] = valid ? part[g] + sbuf[g * kTile + row] : -INFINITY;
+            const float mx = warp_max_f(s[g]);
+            if (lane == 0) red[g * 4 + sub] = mx;
+          }
+          named_barrier(2, 128);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float mt = fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
+            const float m_new = fmaxf(m_run[g], mt);
+            const float alpha = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - m_new);
+            const float pj = valid ? exp2f(s[g] - m_new) : 0.f;
+            P[g * kTile + row] = pj;
+            l_part[g] = l_part[g] * alpha + pj;
+            m_run[g] = m_new;
+            if (row == 0) alpha_s[g] = alpha;
+          }
+        }
+        named_barrier(1, kEpiThreads);
+        // latent-space V accumulation from the staged c_v tile
+        const unsigned char* cvb = sm + p.st_off + stage * p.st_bytes + p.cv_off;
+#pragma unroll
+        for (int vi = 0; vi < 2; ++vi) {
+          const int w = et + vi * kEpiThreads;
+          if (w < p.nv_items) {
+            const int g = w / (rv2 * p.Q);
+            const int rem = w % (rv2 * p.Q);
+            const int q = rem / rv2, m2 = rem % rv2;
+            const float a = alpha_s[g];
+            float o0 = o[vi][0] * a, o1 = o[vi][1] * a;
+            const __nv_bfloat162* cv =
+                reinterpret_cast<const __nv_bfloat162*>(cvb + g * (kTile * p.r_v * 2)) + m2;
+            const float* Pg = P + g * kTile;
+            for (int j = q; j < cnt; j += p.Q) {
+              const float pj = Pg[j];
+              const float2 v = __bfloat1622float2(cv[(size_t)j * rv2]);
+              o0 = fmaf(pj, v.x, o0);
+              o1 = fmaf(pj, v.y, o1);
+            }
+            o[vi][0] = o0;
+            o[vi][1] = o1;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+      }
+      if (aborted) break;
+      // ---------------------------------------------------------- item partial
+      const size_t bh0 = (size_t)r.b * p.H + r.hg * G;
+      if (wgi == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float l = warp_sum_f(l_part[g]);
+          if (lane == 0) red[g * 4 + sub] = l;
+        }
+        named_barrier(2, 128);
+        if (row == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float* part_out = p.partials + ((bh0 + g) * p.S + r.s) * (2 + p.r_v);
+            part_out[0] = m_run[g];
+            part_out[1] = red[g * 4] + red[g * 4 + 1] + red[g * 4 + 2] + red[g * 4 + 3];
+          }
+        }
+      }
+#pragma unroll
+      for (int vi = 0; vi < 2; ++vi) {
+        const int w = et + vi * kEpiThreads;
+        if (w < p.nv_items) {
+          const int g = w / (rv2 * p.Q);
+          const int rem = w % (rv2 * p.Q);
+          const int q = rem / rv2, m2 = rem % rv2;
+          obuf[(q * G + g) * p.r_v + 2 * m2] = o[vi][0];
+          obuf[(q * G + g) * p.r_v + 2 * m2 + 1] = o[vi][1];
+        }
+      }
+      named_barrier(1, kEpiThreads);
+      for (int m = et; m < G * p.r_v; m += kEpiThreads) {
+        const int g = m / p.r_v, mm = m % p.r_v;
+        float acc = 0.f;
+        for (int q = 0; q < p.Q; ++q) acc += obuf[(q * G + g) * p.r_v + mm];
+        p.partials[((bh0 + g) * p.S + r.s) * (2 + p.r_v) + 2 + mm] = acc;
+      }
+      named_barrier(1, kEpiThreads);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* base, int inner, int n_cap, int B, int box_inner,
+              CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)n_cap, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * 2 * n_cap};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)kTile, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* v = std::getenv(name);
+  return v && *v ? std::atoi(v) : dflt;
+}
+
+struct TcPlan {
+  bool ok = false;
+  int G = 1, nst = 0, nacc = 1, S = 0, tps = 0;
+  TcParams p{};
+  uint32_t smem = 0;
+};
+
+// Shared-memory layout for (D, G, nst); returns total bytes (plus alignment slack).
+uint32_t tc_layout(TcParams& p, int D, int G, int nst) {
+  auto al = [](uint32_t x, uint32_t a) { return (x + a - 1) / a * a; };
+  p.K_pad = (p.r_k + 15) / 16 * 16;
+  p.box_k = p.K_pad % 64 == 0 ? 64 : (p.K_pad % 32 == 0 ? 32 : 16);
+  p.nkb = p.K_pad / p.box_k;
+  p.swz = p.box_k == 64 ? 2 : (p.box_k == 32 ? 4 : 6);
+  p.box_bytes = kTile * p.box_k * 2;
+  p.cv_off = G * p.nkb * p.box_bytes;
+  p.st_bytes = al(p.cv_off + G * kTile * p.r_v * 2, 1024);
+  p.tx_bytes = p.cv_off + G * kTile * p.r_v * 2;
+  p.nst = nst;
+  uint32_t o = 0;
+  p.st_off = o;
+  o += nst * p.st_bytes;
+  p.b_off = o;
+  p.b_head_bytes = D * p.K_pad * 2;
+  p.b_sbo = (p.K_pad / 8) * 128;
+  o = al(o + G * p.b_head_bytes, 1024);
+  p.ones_off = o;
+  o += 4096;
+  p.bias_off = o;
+  o = al(o + G * D * 16 * 2, 128);
+  p.qc_off = o;
+  o = al(o + G * (D / 2) * 8, 128);
+  p.sbuf_off = o;
+  o += G * kTile * 4;
+  p.p_off = o;
+  o += G * kTile * 4;
+  p.red_off = o;
+  o += G * 4 * 4;
+  p.alpha_off = o;
+  o = al(o + G * 4, 16);
+  const int rv2 = p.r_v / 2;
+  int Q = kEpiThreads / (G * rv2);
+  if (Q < 1) Q = 1;
+  if (Q > 8) Q = 8;
+  p.Q = Q;
+  p.nv_items = G * rv2 * Q;
+  p.obuf_off = o;
+  o = al(o + Q * G * p.r_v * 4, 16);
+  p.bar_off = o;
+  o += (2 * nst + 5) * 8;
+  p.misc_off = o;
+  o += 16;
+  return o + 1024;
+}
+
+TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
+  TcPlan pl;
+  const int D = c.d_head;
+  if (c.mode != LLA_MODE_PER_HEAD || n_cap <= 0 || B <= 0) return pl;
+  if (D != 32 && D != 64 && D != 96 && D != 128) return pl;
+  const int forced_g = env_int("LLA_TC_G", 0), forced_nst = env_int("LLA_TC_NST", 0);
+  // Largest head group G whose ring fits at least 3 stages; else the largest with 2.
+  int best_g = 0, best_nst = 0;
+  for (int G : {4, 2, 1}) {
+    if (c.H % G || G * D > 512) continue;
+    if (forced_g && G != forced_g) continue;
+    TcParams p{};
+    p.r_k = c.r_k;
+    p.r_v = c.r_v;
+    int nst = 0;
+    for (int s = 2; s <= 6; ++s)
+      if (tc_layout(p, D, G, s) <= kSmemLimit) nst = s;
+    if (forced_nst && nst > forced_nst) nst = forced_nst;
+    if (nst >= 3) {
+      best_g = G;
+      best_nst = nst;
+      break;
+    }
+    if (nst >= 2 && best_g == 0) {
+      best_g = G;
+      best_nst = nst;
+    }
+  }
+  if (!best_g) return pl;
+  pl.G = best_g;
+  pl.nst = best_nst;
+  pl.nacc = (2 * pl.G * D <= 512) ? 2 : 1;
+  // Context splits: balance tiles over a 148-SM grid of persistent CTAs.
+  const int n_tiles = (n_cap + kTile - 1) / kTile;
+  const long long units = (long long)B * (c.H / pl.G);
+  const int grid = 148;
+  double best_eff = -1.0;
+  int best_s = 1;
+  for (int S = 1; S <= kMaxSplits && S <= n_tiles; ++S) {
+    const int tpi = (n_tiles + S - 1) / S;
+    const int s_eff = (n_tiles + tpi - 1) / tpi;
+    const long long items = units * s_eff;
+    const long long per_cta = (items + grid - 1) / grid * tpi;
+    const double eff = (double)units * n_tiles / ((double)grid * per_cta);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best_s = s_eff;
+    }
+    if (eff >= 0.93) break;
+  }
+  pl.tps = (n_tiles + best_s - 1) / best_s;
+  pl.S = (n_tiles + pl.tps - 1) / pl.tps;
+  pl.ok = true;
+  return pl;
+}
+
+bool tc_enabled() {
+  const char* v = std::getenv("LLA_DECODE_PATH");
+  return !(v && std::strcmp(v, "cuda_core") == 0);
+}
+
+template <int D, int G>
+cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
+                        uint32_t smem, int grid, cudaStream_t s) {
+  auto kern = decode_tc_kernel<D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, s>>>(mk, mv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_tc_d(int G, const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
+                        uint32_t smem, int grid, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_tc_t<D, 1>(mk, mv, p, smem, grid, s);
+    case 2: return launch_tc_t<D, 2>(mk, mv, p, smem, grid, s);
+    case 4: return launch_tc_t<D, 4>(mk, mv, p, smem, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps) {
+  if (!tc_enabled()) return false;
+  TcPlan pl = tc_plan(c, B, n_cap);
+  if (!pl.ok) return false;
+  *S = pl.S;
+  *tps = pl.tps;
+  return true;
+}
+
+// Launch the tensor-core partial kernel; returns cudaErrorNotSupported when the
+// shape is outside this path (the caller then uses the CUDA-core kernel).
+cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t s) {
+  if (!tc_enabled()) return cudaErrorNotSupported;
+  TcPlan pl = tc_plan(c, a.B, a.n_cap);
+  if (!pl.ok || pl.S != a.S) return cudaErrorNotSupported;
+  TcParams p{};
+  p.H = a.H;
+  p.r_k = a.r_k;
+  p.r_v = a.r_v;
+  // At least 120 KB so that two CTAs never share an SM (each may hold all of TMEM).
+  uint32_t smem = tc_layout(p, a.d, pl.G, pl.nst);
+  if (smem < 120u * 1024u) smem = 120u * 1024u;
+  p.B = a.B;
+  p.n_cap = a.n_cap;
+  p.S = pl.S;
+  p.tps = pl.tps;
+  p.HG = a.H / pl.G;
+  p.n_items = a.B * p.HG * pl.S;
+  p.rope_max_pos = a.rope_max_pos;
+  p.kappa = a.kappa;
+  p.nacc = pl.nacc;
+  p.acc_cols = pl.G * a.d;
+  int cols = 32;
+  while (cols < p.nacc * p.acc_cols) cols <<= 1;
+  p.tmem_cols = cols;
+  p.wupk_t = a.wupk_t;
+  p.muk_t = a.muk_t;
+  p.rope = a.rope;
+  p.ctx_len = a.ctx_len;
+  p.q = a.q;
+  p.positions = a.positions;
+  p.q_pos = a.q_pos;
+  p.status = a.status;
+  p.partials = a.partials;
+  CUtensorMap mk, mv;
+  const CUtensorMapSwizzle swz = p.box_k == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!make_map(&mk, a.ck, a.H * a.r_k, a.n_cap, a.B, p.box_k, swz) ||
+      !make_map(&mv, a.cv, a.H * a.r_v, a.n_cap, a.B, a.r_v, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorNotSupported;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  switch (a.d) {
+    case 32: return launch_tc_d<32>(pl.G, mk, mv, p, smem, grid, s);
+    case 64: return launch_tc_d<64>(pl.G, mk, mv, p, smem, grid, s);
+    case 96: return launch_tc_d<96>(pl.G, mk, mv, p, smem, grid, s);
+    case 128: return launch_tc_d<128>(pl.G, mk, mv, p, smem, grid, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace lla

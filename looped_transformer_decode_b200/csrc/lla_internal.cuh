@@ -36,6 +36,7 @@ struct SplitPlan {
   int n_tiles;          // ceil(n_cap / kTile)
   int splits;           // S
   int tiles_per_split;  // tiles handled by one CTA
+  bool tensor_cores;    // the tcgen05 partial kernel takes this shape
 };
 SplitPlan split_plan(const lla_cfg& c, int B, int n_cap);
 size_t partials_bytes(const lla_cfg& c, int B, int S);
@@ -75,6 +76,13 @@ struct DecodeArgs {
   int S, tiles_per_split;
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
+
+// Tensor-core (tcgen05) partial kernel for per-head decode.  decode_tc_plan
+// reports whether the shape takes that path and its context split; the launcher
+// returns cudaErrorNotSupported when it cannot run the shape.
+bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps);
+cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t s);
 
 // Record `fmt` as the calling thread's lla_last_error() message; returns `code`.
 int set_error(int code, const char* fmt, ...);

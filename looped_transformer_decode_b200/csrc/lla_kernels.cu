@@ -463,9 +463,14 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches) {
     if (e != cudaSuccess) return e;
     ++*launches;
   }
+  cudaError_t e = launch_combine(a, s);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
   dim3 g2((unsigned)a.H, (unsigned)a.B);
   decode_combine_kernel<<<g2, 128, 0, s>>>(a);
-  ++*launches;
   return cudaGetLastError();
 }
 
