@@ -106,10 +106,12 @@ SplitPlan split_plan(const lla_cfg& c, int B, int n_cap) {
     return p;
   }
   int S_tc = 0, tps_tc = 0;
-  if (decode_tc_plan(c, B, n_cap, &S_tc, &tps_tc)) {
+  size_t ops = 0;
+  if (decode_tc_plan(c, B, n_cap, &S_tc, &tps_tc, &ops)) {
     p.splits = S_tc;
     p.tiles_per_split = tps_tc;
     p.tensor_cores = true;
+    p.ops_bytes = ops;
     return p;
   }
   // Aim for about four resident CTAs per SM on a 148-SM part.
@@ -253,13 +255,14 @@ size_t lla_decode_workspace_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap) 
   if (check_cfg(cfg) || B < 0 || n_cap < 0) return 0;
   ok();
   SplitPlan p = split_plan(*cfg, B, n_cap);
-  return kWsHeader + partials_bytes(*cfg, B, p.splits);
+  return kWsHeader + align_up(partials_bytes(*cfg, B, p.splits), 256) + p.ops_bytes;
 }
 
 int lla_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap) {
   if (check_cfg(cfg) || B < 0 || n_cap < 0) return -1;
   if (B == 0) return 0;
-  return n_cap > 0 ? 2 : 1;
+  if (n_cap == 0) return 1;
+  return split_plan(*cfg, B, n_cap).tensor_cores ? 3 : 2;
 }
 
 int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_table,
@@ -289,7 +292,7 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
     }
   }
   SplitPlan plan = split_plan(*cfg, B, n_cap);
-  size_t need = kWsHeader + partials_bytes(*cfg, B, plan.splits);
+  size_t need = kWsHeader + align_up(partials_bytes(*cfg, B, plan.splits), 256) + plan.ops_bytes;
   if (ws_bytes < need)
     return fail(LLA_ERR_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
 
@@ -309,6 +312,7 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   a.B = B;
   a.n_cap = n_cap;
   a.rope_max_pos = rope_max_pos;
+  a.rope_base = cfg->rope_base;
   a.wupk_t = reinterpret_cast<const float*>(pk + L.wupk) + (size_t)t * H * d * cfg->r_k;
   a.wupv_t = reinterpret_cast<const float*>(pk + L.wupv) + (size_t)t * H * d * cfg->r_v;
   a.muk_t = reinterpret_cast<const float*>(pk + L.muk) + (size_t)t * H * d;
@@ -338,6 +342,10 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   a.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
   a.S = plan.splits;
   a.tiles_per_split = plan.tiles_per_split;
+  a.ops = plan.tensor_cores
+              ? static_cast<unsigned char*>(ws) + kWsHeader +
+                    align_up(partials_bytes(*cfg, B, plan.splits), 256)
+              : nullptr;
   int launches = 0;
   cudaError_t ce = cudaErrorNotSupported;
   if (plan.tensor_cores && plan.splits > 0) {

@@ -38,30 +38,59 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;       // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
-constexpr int kEpiThreads = 256;
+constexpr int kEpiWG = 2;                       // epilogue warpgroups
+constexpr int kEpiThreads = 128 * kEpiWG;       // warps 2 .. 2 + 4 kEpiWG - 1
+constexpr int kEpiWarps = kEpiThreads / 32;
+constexpr int kThreads = 64 + kEpiThreads;      // warp 0 TMA, warp 1 MMA, then the epilogue
 constexpr uint32_t kSmemLimit = 232448;  // per-block dynamic shared memory on sm_100
 
 struct TcParams {
   int H, r_k, r_v, K_pad, box_k, nkb, swz;   // swz: descriptor swizzle code
   int Q, nv_items;                           // V-phase split: token residues, work items
   int B, n_cap, S, tps, HG, n_items, rope_max_pos;
-  float kappa;
   uint32_t st_off, st_bytes, cv_off, box_bytes;
-  uint32_t b_off, b_head_bytes, b_sbo, ones_off, bias_off, qc_off, sbuf_off, p_off, red_off,
-      alpha_off, obuf_off, bar_off, misc_off;
+  uint32_t b_off, b_head_bytes, b_sbo, bias_head_bytes, ones_off, bias_off, sbuf_off, p_off,
+      red_off, alpha_off, obuf_off, bar_off, misc_off;
   int nst, nacc, acc_cols, tmem_cols;
   uint32_t tx_bytes;
-  const float* wupk_t;   // [H][d][r_k]
-  const float* muk_t;    // [H][d]
   const float2* rope;    // [rope_max_pos][d/2]
   const int32_t* ctx_len;
-  const float* q;        // [B][H][d]
   const int32_t* positions;
-  const int32_t* q_pos;
+  const unsigned char* ops_b;     // [B][H] images of the MMA B operand
+  const unsigned char* ops_bias;  // [B][H] images of the bias tile
   int32_t* status;
   float* partials;       // [B][H][S][2 + r_v]
+  // theta_i / (2 pi) as 64-bit fixed-point fractions of a turn, per RoPE pair i
+  uint32_t phi_lo[64], phi_hi[64];
+  // conj(e^{i 128 theta_i}): advances conj(e^{i p theta_i}) by one tile of positions
+  float2 step[64];
 };
+
+constexpr int kNoPos = -2147483647 - 1;       // raw position of a row past the context
+constexpr int kReseedTiles = 32;              // exact RoPE factors at least this often
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long ra, rb, rc, rd;
+  memcpy(&ra, &a, 8);
+  memcpy(&rb, &b, 8);
+  memcpy(&rc, &c, 8);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
+  float2 d;
+  memcpy(&d, &rd, 8);
+  return d;
+}
+
+// (cos, -sin) of pos * theta_i, i.e. conj(e^{i pos theta_i}).  The angle is reduced exactly in integer arithmetic
+// (pos * phi_i mod 1 turn, phi_i = theta_i / 2pi in 0.64 fixed point), so the
+// fp32 sine and cosine see an argument in [-pi, pi) with error below 1e-7 rad at
+// any position.
+__device__ __forceinline__ float2 rope_factor(uint32_t pos, uint32_t phi_lo, uint32_t phi_hi) {
+  const uint32_t turns = pos * phi_hi + __umulhi(pos, phi_lo);
+  const float ang = static_cast<float>(static_cast<int32_t>(turns)) * 1.46291807926715968e-9f;
+  float sn, cs;
+  __sincosf(ang, &sn, &cs);
+  return make_float2(cs, -sn);
+}
 
 __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
@@ -75,18 +104,30 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
-// bar.red.or over the 256 epilogue threads (named barrier 1): returns the OR of `pred`.
+// bar.red.or over the epilogue threads (named barrier 1): returns the OR of `pred`.
 __device__ __forceinline__ int epi_barrier_or(int pred) {
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "barrier.red.or.pred po, 1, 256, pi;\n\t"
+      "barrier.red.or.pred po, 1, %2, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}\n"
       : "=r"(out)
-      : "r"(pred)
+      : "r"(pred), "n"(kEpiThreads)
       : "memory");
   return static_cast<int>(out);
+}
+
+// TMEM -> registers, 8 consecutive columns (32x32b shape).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 struct ItemRange {
@@ -110,61 +151,120 @@ __device__ __forceinline__ ItemRange item_range(const TcParams& p, int item, boo
   return r;
 }
 
-// Rebuild the MMA B operand A~ (no-swizzle K-major, rows n = 2i (Re) / 2i+1 (Im))
-// and the bias tile for item (b, head group) in shared memory.  All 256 epilogue
-// threads take part; ends with the proxy fence and an epilogue barrier.
-template <int D, int G>
-__device__ void prepare_item(const TcParams& p, unsigned char* sm, int et, int b, int hg) {
+// Walks this CTA's tiles in processing order (items with no tiles are skipped).
+struct TileCursor {
+  int item, k;
+  ItemRange r;
+  bool valid;
+};
+
+__device__ __forceinline__ void cursor_first(const TcParams& p, TileCursor& c) {
+  c.valid = false;
+  c.k = 0;
+  for (c.item = blockIdx.x; c.item < p.n_items; c.item += gridDim.x) {
+    c.r = item_range(p, c.item, false);
+    if (c.r.ntiles > 0) {
+      c.valid = true;
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void cursor_next(const TcParams& p, TileCursor& c) {
+  if (!c.valid) return;
+  if (++c.k < c.r.ntiles) return;
+  c.k = 0;
+  for (c.item += gridDim.x; c.item < p.n_items; c.item += gridDim.x) {
+    c.r = item_range(p, c.item, false);
+    if (c.r.ntiles > 0) return;
+  }
+  c.valid = false;
+}
+
+// Raw position of token `row` of the cursor's tile (0 for rows past the context).
+// The range check is left to the consumer so that the load does not stall here.
+__device__ __forceinline__ int cursor_pos(const TcParams& p, const TileCursor& c, int row) {
+  if (!c.valid) return kNoPos;
+  const int t0 = c.r.tok0 + c.k * kTile;
+  if (row >= c.r.tok_end - t0) return kNoPos;
+  return p.positions[(size_t)c.r.b * p.n_cap + t0 + row];
+}
+
+__device__ __forceinline__ int checked_pos(const TcParams& p, int pos) {
+  if (pos < 0 || pos >= p.rope_max_pos) {
+    atomicOr(p.status, LLA_STATUS_POSITION_RANGE);
+    return 0;
+  }
+  return pos;
+}
+
+// Builds, for every (b, h), the MMA B operand A~ (rows n = 2i: Re, 2i+1: Im of the
+// query-absorbed up-projection, K = latent index) as the byte image of the
+// no-swizzle K-major shared-memory layout, and the bias tile image (K column 0 =
+// bf16 hi part of M~, column 1 = lo part).  One CTA of 128 threads per (h, b).
+template <int D>
+__global__ void __launch_bounds__(128) decode_prep_kernel(
+    const float* __restrict__ q, const int32_t* __restrict__ q_pos, const float2* __restrict__ rope,
+    int rope_max_pos, const float* __restrict__ wupk_t, const float* __restrict__ muk_t, float kappa,
+    int H, int r_k, int K_pad, unsigned char* __restrict__ ops_b,
+    unsigned char* __restrict__ ops_bias, int32_t* status) {
   constexpr int HALF = D / 2;
-  float2* qc = reinterpret_cast<float2*>(sm + p.qc_off);
-  int qp = p.q_pos[b];
-  if (qp < 0 || qp >= p.rope_max_pos) {
-    if (et == 0) atomicOr(p.status, LLA_STATUS_POSITION_RANGE);
+  __shared__ float2 qc[HALF];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  int qp = q_pos[b];
+  if (qp < 0 || qp >= rope_max_pos) {
+    if (tid == 0 && h == 0 && blockIdx.z == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
     qp = 0;
   }
-  for (int idx = et; idx < G * HALF; idx += kEpiThreads) {
-    const int g = idx / HALF, i = idx % HALF;
-    const int h = hg * G + g;
-    const float2 e = p.rope[(size_t)qp * HALF + i];
-    const float* qh = p.q + ((size_t)b * p.H + h) * D;
+  const float* qh = q + ((size_t)b * H + h) * D;
+  for (int i = tid; i < HALF; i += blockDim.x) {
+    const float2 e = rope[(size_t)qp * HALF + i];
     const float x0 = qh[i], x1 = qh[i + HALF];
-    qc[idx] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
+    qc[i] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
   }
-  named_barrier(1, kEpiThreads);
-  const int Kp = p.K_pad;
-  for (int idx = et; idx < G * D * Kp; idx += kEpiThreads) {
-    const int k = idx % Kp;
-    const int n = (idx / Kp) % D;
-    const int g = idx / (D * Kp);
-    const int h = hg * G + g;
+  __syncthreads();
+  const float* W = wupk_t + (size_t)h * D * r_k;  // [d][r_k]
+  unsigned char* img = ops_b + ((size_t)b * H + h) * (size_t)D * K_pad * 2;
+  // One 16-byte chunk (8 consecutive K values of one row n) per iteration.
+  const int chunks = D * K_pad / 8;
+  for (int c = blockIdx.z * blockDim.x + tid; c < chunks; c += gridDim.z * blockDim.x) {
+    const int n = (c / K_pad) * 8 + (c & 7);
+    const int k0 = ((c >> 3) % (K_pad / 8)) * 8;
     const int i = n >> 1;
-    float val = 0.f;
-    if (k < p.r_k) {
-      const float* W = p.wupk_t + (size_t)h * D * p.r_k;
-      const float wr = W[(size_t)i * p.r_k + k], wi = W[(size_t)(i + HALF) * p.r_k + k];
-      const float2 z = qc[g * HALF + i];
-      val = (n & 1) ? p.kappa * (z.x * wi - z.y * wr) : p.kappa * (z.x * wr + z.y * wi);
+    const float2 z = qc[i];
+    __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = k0 + e;
+      float val = 0.f;
+      if (k < r_k) {
+        const float wr = W[(size_t)i * r_k + k], wi = W[(size_t)(i + HALF) * r_k + k];
+        val = (n & 1) ? kappa * (z.x * wi - z.y * wr) : kappa * (z.x * wr + z.y * wi);
+      }
+      v[e] = __float2bfloat16_rn(val);
     }
-    const uint32_t off = p.b_off + g * p.b_head_bytes + (n >> 3) * p.b_sbo + (k >> 3) * 128 +
-                         (n & 7) * 16 + (k & 7) * 2;
-    *reinterpret_cast<__nv_bfloat16*>(sm + off) = __float2bfloat16_rn(val);
+    *reinterpret_cast<uint4*>(img + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
   }
-  for (int idx = et; idx < G * D; idx += kEpiThreads) {
-    const int n = idx % D, g = idx / D;
-    const int h = hg * G + g;
-    const int i = n >> 1;
-    const float* mu = p.muk_t + (size_t)h * D;
-    const float mr = mu[i], mi = mu[i + HALF];
-    const float2 z = qc[g * HALF + i];
-    const float val = (n & 1) ? p.kappa * (z.x * mi - z.y * mr) : p.kappa * (z.x * mr + z.y * mi);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(val);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
-    const uint32_t off = p.bias_off + g * (D * 16 * 2) + (n >> 3) * 256 + (n & 7) * 16;
-    *reinterpret_cast<__nv_bfloat16*>(sm + off) = hi;
-    *reinterpret_cast<__nv_bfloat16*>(sm + off + 2) = lo;
+  // Bias tile image [D x 16]: chunk c covers row n = (c / 2 / 8) * 8 + c % 8 ... laid out as
+  // core matrices (n / 8, k / 8) at (n / 8) * 256 + (k / 8) * 128 + (n % 8) * 16.
+  unsigned char* bimg = ops_bias + ((size_t)b * H + h) * (size_t)D * 32;
+  const float* mu = muk_t + (size_t)h * D;
+  for (int c = blockIdx.z * blockDim.x + tid; c < D * 2; c += gridDim.z * blockDim.x) {
+    const int n = (c >> 4) * 8 + (c & 7);
+    const int kc = (c >> 3) & 1;
+    __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __float2bfloat16_rn(0.f);
+    if (kc == 0) {
+      const int i = n >> 1;
+      const float2 z = qc[i];
+      const float mr = mu[i], mi = mu[i + HALF];
+      const float val = (n & 1) ? kappa * (z.x * mi - z.y * mr) : kappa * (z.x * mr + z.y * mi);
+      v[0] = __float2bfloat16_rn(val);
+      v[1] = __float2bfloat16_rn(val - __bfloat162float(v[0]));
+    }
+    *reinterpret_cast<uint4*>(bimg + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
   }
-  fence_proxy_async_smem();
-  named_barrier(1, kEpiThreads);
 }
 
 template <int D, int G>
@@ -172,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
   constexpr int HALF = D / 2;
-  constexpr int WG_PAIRS = D / 4;   // RoPE pairs per epilogue warpgroup
+  constexpr int WG_PAIRS = HALF / kEpiWG;   // RoPE pairs per epilogue warpgroup
+  constexpr int WG_COLS = 2 * WG_PAIRS;     // TMEM columns per warpgroup (Re, Im interleaved)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -180,22 +281,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + p.nst;
   uint64_t* tfull = empty + p.nst;
   uint64_t* tempty = tfull + 2;
-  uint64_t* bop = tempty + 2;
+  uint64_t* bfull = tempty + 2;    // [2] B operand buffers loaded
+  uint64_t* bempty = bfull + 2;    // [2] B operand buffers free (MMAs done)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ops_head_bytes = p.b_head_bytes;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 8);
+      mbar_init(&empty[s], kEpiWarps);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);
+      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&bfull[a], 1);
+      mbar_init(&bempty[a], 1);
     }
-    mbar_init(bop, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -205,14 +309,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp >= 2) {
     const int et = threadIdx.x - 64;
-    // ones tile [128 x 16]: columns 0 and 1 hold 1.0; bias tiles start at zero.
+    // ones tile [128 x 16]: columns 0 and 1 hold 1.0 (adds bias hi + lo to every row).
     for (int idx = et; idx < 128 * 16; idx += kEpiThreads) {
       const int m = idx / 16, k = idx % 16;
       const uint32_t off = p.ones_off + (m >> 3) * 256 + (k >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2;
       *reinterpret_cast<__nv_bfloat16*>(sm + off) = __float2bfloat16_rn(k < 2 ? 1.f : 0.f);
     }
-    for (int idx = et; idx < G * D * 16; idx += kEpiThreads)
-      reinterpret_cast<__nv_bfloat16*>(sm + p.bias_off)[idx] = __float2bfloat16_rn(0.f);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -224,10 +327,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&map_k);
       tma_prefetch_desc(&map_v);
-      uint32_t it = 0;
+      uint32_t it = 0, jn = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, item, false);
+        if (r.ntiles == 0) continue;
+        {
+          // query-absorbed operands of this item into B buffer jn & 1
+          const uint32_t buf = jn & 1u, bph = (jn >> 1) & 1u;
+          if (!mbar_wait(&bempty[buf], bph ^ 1u, abort_flag)) break;
+          const size_t head0 = (size_t)r.b * p.H + (size_t)r.hg * G;
+          mbar_arrive_expect_tx(&bfull[buf], G * (ops_head_bytes + p.bias_head_bytes));
+          bulk_load(sm + p.b_off + buf * G * ops_head_bytes, p.ops_b + head0 * ops_head_bytes,
+                    G * ops_head_bytes, &bfull[buf]);
+          bulk_load(sm + p.bias_off + buf * G * p.bias_head_bytes,
+                    p.ops_bias + head0 * p.bias_head_bytes, G * p.bias_head_bytes, &bfull[buf]);
+          ++jn;
+        }
         for (int k = 0; k < r.ntiles; ++k, ++it) {
           const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
           if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) {
@@ -248,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
+      if (*abort_flag) {
         // Drain: wait (bounded) for every copy this thread issued before leaving.
         const uint32_t n_out = it < (uint32_t)p.nst ? it : (uint32_t)p.nst;
         for (uint32_t j = 0; j < n_out; ++j) {
@@ -258,6 +374,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           while (!mbar_try_wait(&full[stage], ph) && global_timer_ns() - t0 < kWaitTimeoutNs) {
           }
         }
+        for (uint32_t j = 0; j < 2 && j < jn; ++j) {
+          const uint32_t i = jn - 1 - j;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&bfull[i & 1u], (i >> 1) & 1u) &&
+                 global_timer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
       }
     }
   } else if (warp == 1) {
@@ -265,15 +388,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D);
       const uint32_t sbo_a = 16u * p.box_k;
-      const uint32_t ones_addr = smem_addr(sm + p.ones_off);
-      uint32_t it = 0, item_no = 0;
+      const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 256, 0);
+      uint32_t it = 0, jn = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, item, false);
-        if (r.ntiles == 0) continue;   // no tiles: the epilogue prepares nothing either
-        if (!mbar_wait(bop, item_no & 1u, abort_flag)) break;
-        ++item_no;
-        tc_fence_after();
+        if (r.ntiles == 0) continue;
+        const uint32_t buf = jn & 1u, bph = (jn >> 1) & 1u;
+        if (!mbar_wait(&bfull[buf], bph, abort_flag)) break;
+        ++jn;
+        const uint32_t b_base = smem_addr(sm + p.b_off + buf * G * ops_head_bytes);
+        const uint32_t bias_base = smem_addr(sm + p.bias_off + buf * G * p.bias_head_bytes);
         for (int k = 0; k < r.ntiles; ++k, ++it) {
           const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
           const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
@@ -287,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const uint32_t d_tmem = tmem_base + acc * p.acc_cols + g * D;
-            const uint32_t b_addr = smem_addr(sm + p.b_off + g * p.b_head_bytes);
+            const uint32_t b_addr = b_base + g * ops_head_bytes;
             for (int kk = 0; kk < p.K_pad / 16; ++kk) {
               const int kb = (kk * 16) / p.box_k, kin = (kk * 16) % p.box_k;
               const uint64_t adesc =
@@ -295,66 +420,83 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t bdesc = smem_desc(b_addr + kk * 256, 128, p.b_sbo, 0);
               mma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
             }
-            const uint64_t odesc = smem_desc(ones_addr, 128, 256, 0);
-            const uint64_t bias_desc =
-                smem_desc(smem_addr(sm + p.bias_off + g * (D * 16 * 2)), 128, 256, 0);
+            const uint64_t bias_desc = smem_desc(bias_base + g * p.bias_head_bytes, 128, 256, 0);
             mma_bf16(d_tmem, odesc, bias_desc, idesc, 1u);
           }
           mma_commit(&tfull[acc]);
         }
+        if (ok) mma_commit(&bempty[buf]);   // B buffer reusable once these MMAs finish
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;
-    const int wgi = (warp - 2) >> 2;          // which half of the RoPE pairs
+    const int wgi = (warp - 2) >> 2;          // which quarter of the RoPE pairs
     const int sub = warp & 3;                 // TMEM sub-partition of this warp
     const int row = sub * 32 + lane;          // token row of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
-    float* sbuf = reinterpret_cast<float*>(sm + p.sbuf_off);   // [G][128]
+    float* sbuf = reinterpret_cast<float*>(sm + p.sbuf_off);   // [kEpiWG - 1][G][128]
     float* P = reinterpret_cast<float*>(sm + p.p_off);         // [G][128]
     float* red = reinterpret_cast<float*>(sm + p.red_off);     // [G][4]
     float* alpha_s = reinterpret_cast<float*>(sm + p.alpha_off);
     float* obuf = reinterpret_cast<float*>(sm + p.obuf_off);   // [Q][G][r_v]
-    const int rv2 = p.r_v >> 1;
+    const int rv8 = p.r_v >> 3;
+
+    // Software pipeline of the RoPE factors: the table row of tile it+1 is loaded
+    // while tile it is processed, and positions two tiles ahead.
+    TileCursor pc;
+    cursor_first(p, pc);
+    // conj(e^{i p theta_i}) for this thread's RoPE pairs at position pos_cur of its
+    // token; when the next tile's token sits exactly one tile further on, the
+    // factors advance by one complex product, otherwise they are recomputed.
+    float2 ef[WG_PAIRS];
+    int pos_cur = kNoPos, run = 0;
+    auto advance_rope = [&](int praw) {
+      if (praw == kNoPos) return;               // row past the context: keep factors
+      const int pn = checked_pos(p, praw);
+      if (pos_cur != kNoPos && pn == pos_cur + kTile && run < kReseedTiles) {
+#pragma unroll
+        for (int q = 0; q < WG_PAIRS; ++q) {
+          const float2 st = p.step[wgi * WG_PAIRS + q];
+          const float2 e = ef[q];
+          ef[q] = make_float2(fmaf(e.x, st.x, -e.y * st.y), fmaf(e.x, st.y, e.y * st.x));
+        }
+        ++run;
+      } else {
+#pragma unroll
+        for (int q = 0; q < WG_PAIRS; ++q)
+          ef[q] = rope_factor(static_cast<uint32_t>(pn), p.phi_lo[wgi * WG_PAIRS + q],
+                              p.phi_hi[wgi * WG_PAIRS + q]);
+        run = 0;
+      }
+      pos_cur = pn;
+    };
+#pragma unroll
+    for (int q = 0; q < WG_PAIRS; ++q) ef[q] = make_float2(1.f, 0.f);
+    advance_rope(cursor_pos(p, pc, row));
+    cursor_next(p, pc);
+    int pos_next = cursor_pos(p, pc, row);
+    cursor_next(p, pc);
 
     uint32_t it = 0;
     bool aborted = false;
     for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
       const ItemRange r = item_range(p, item, et == 0);
-      if (r.ntiles > 0) {
-        // The previous item's MMAs have all completed (its last tile was read from
-        // TMEM), so the B operand can be rebuilt; one arrival per non-empty item.
-        prepare_item<D, G>(p, sm, et, r.b, r.hg);
-        if (et == 0) mbar_arrive(bop);
-      }
       float m_run[G], l_part[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         m_run[g] = -INFINITY;
         l_part[g] = 0.f;
       }
-      float o[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      float2 o[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                     make_float2(0.f, 0.f)};
       for (int k = 0; k < r.ntiles; ++k, ++it) {
         const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
         const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
         const int t0 = r.tok0 + k * kTile;
         const int cnt = min(kTile, r.tok_end - t0);
         const bool valid = row < cnt;
-        int pos = 0;
-        if (valid) {
-          pos = p.positions[(size_t)r.b * p.n_cap + t0 + row];
-          if (pos < 0 || pos >= p.rope_max_pos) {
-            atomicOr(p.status, LLA_STATUS_POSITION_RANGE);
-            pos = 0;
-          }
-        }
-        float4 e4[WG_PAIRS / 2];
-        const float4* erow =
-            reinterpret_cast<const float4*>(p.rope + (size_t)pos * HALF + wgi * WG_PAIRS);
-#pragma unroll
-        for (int c = 0; c < WG_PAIRS / 2; ++c) e4[c] = erow[c];
 
         bool ok = mbar_wait(&tfull[acc], aph, abort_flag);
         tc_fence_after();
@@ -362,27 +504,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           part[g] = 0.f;
-          const uint32_t col = tmem_base + lane_addr + acc * p.acc_cols + g * D + wgi * HALF;
-          float u[HALF];
+          const uint32_t col = tmem_base + lane_addr + acc * p.acc_cols + g * D + wgi * WG_COLS;
+          float u[WG_COLS];
 #pragma unroll
-          for (int c = 0; c < HALF / 16; ++c) tmem_ld16(col + c * 16, u + c * 16);
+          for (int c = 0; c < WG_COLS / 16; ++c) tmem_ld16(col + c * 16, u + c * 16);
+          if constexpr (WG_COLS % 16 != 0) tmem_ld8(col + (WG_COLS / 16) * 16, u + (WG_COLS / 16) * 16);
           tmem_wait_ld();
+          float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int q2 = 0; q2 < HALF / 4; ++q2) {
-            const float4 e = e4[q2];   // (cos, sin) of two consecutive pairs
-            part[g] = fmaf(u[4 * q2], e.x, part[g]);
-            part[g] = fmaf(-u[4 * q2 + 1], e.y, part[g]);
-            part[g] = fmaf(u[4 * q2 + 2], e.z, part[g]);
-            part[g] = fmaf(-u[4 * q2 + 3], e.w, part[g]);
-          }
+          for (int q = 0; q < WG_PAIRS; ++q) acc2 = ffma2(make_float2(u[2 * q], u[2 * q + 1]), ef[q], acc2);
+          part[g] = acc2.x + acc2.y;
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
+        // RoPE factors of the next tile (its position was loaded a tile ago), and
+        // the raw position of the tile after it
+        advance_rope(pos_next);
+        pos_next = cursor_pos(p, pc, row);
+        cursor_next(p, pc);
         ok = ok && mbar_wait(&full[stage], ph, abort_flag);
-        if (wgi == 1) {
+        if (wgi > 0) {
 #pragma unroll
-          for (int g = 0; g < G; ++g) sbuf[g * kTile + row] = part[g];
+          for (int g = 0; g < G; ++g) sbuf[((wgi - 1) * G + g) * kTile + row] = part[g];
         }
         if (epi_barrier_or(!ok)) {
           aborted = true;
@@ -392,7 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float s[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            s[g] = valid ? part[g] + sbuf[g * kTile + row] : -INFINITY;
+            float tot = part[g];
+#pragma unroll
+            for (int w = 0; w < kEpiWG - 1; ++w) tot += sbuf[(w * G + g) * kTile + row];
+            s[g] = valid ? tot : -INFINITY;
             const float mx = warp_max_f(s[g]);
             if (lane == 0) red[g * 4 + sub] = mx;
           }
@@ -410,28 +557,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         named_barrier(1, kEpiThreads);
-        // latent-space V accumulation from the staged c_v tile
-        const unsigned char* cvb = sm + p.st_off + stage * p.st_bytes + p.cv_off;
+        // latent-space V accumulation from the staged c_v tile: thread = (head,
+        // 8 latent dims, token residue q); tokens j = q, q + Q, ...
+        if (et < p.nv_items) {
+          const unsigned char* cvb = sm + p.st_off + stage * p.st_bytes + p.cv_off;
+          const int g = et / (rv8 * p.Q);
+          const int rem = et % (rv8 * p.Q);
+          const int q = rem / rv8, c8 = rem % rv8;
+          const float a = alpha_s[g];
 #pragma unroll
-        for (int vi = 0; vi < 2; ++vi) {
-          const int w = et + vi * kEpiThreads;
-          if (w < p.nv_items) {
-            const int g = w / (rv2 * p.Q);
-            const int rem = w % (rv2 * p.Q);
-            const int q = rem / rv2, m2 = rem % rv2;
-            const float a = alpha_s[g];
-            float o0 = o[vi][0] * a, o1 = o[vi][1] * a;
-            const __nv_bfloat162* cv =
-                reinterpret_cast<const __nv_bfloat162*>(cvb + g * (kTile * p.r_v * 2)) + m2;
-            const float* Pg = P + g * kTile;
-            for (int j = q; j < cnt; j += p.Q) {
-              const float pj = Pg[j];
-              const float2 v = __bfloat1622float2(cv[(size_t)j * rv2]);
-              o0 = fmaf(pj, v.x, o0);
-              o1 = fmaf(pj, v.y, o1);
-            }
-            o[vi][0] = o0;
-            o[vi][1] = o1;
+          for (int e = 0; e < 4; ++e) o[e] = make_float2(o[e].x * a, o[e].y * a);
+          const uint4* cv = reinterpret_cast<const uint4*>(cvb + g * (kTile * p.r_v * 2)) + c8;
+          const float* Pg = P + g * kTile;
+#pragma unroll 2
+          for (int j = q; j < cnt; j += p.Q) {
+            const float pj = Pg[j];
+            const float2 pj2 = make_float2(pj, pj);
+            const uint4 raw = cv[(size_t)j * rv8];
+            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = ffma2(pj2, __bfloat1622float2(v2[e]), o[e]);
           }
         }
         __syncwarp();
@@ -456,15 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (et < p.nv_items) {
+        const int g = et / (rv8 * p.Q);
+        const int rem = et % (rv8 * p.Q);
+        const int q = rem / rv8, c8 = rem % rv8;
 #pragma unroll
-      for (int vi = 0; vi < 2; ++vi) {
-        const int w = et + vi * kEpiThreads;
-        if (w < p.nv_items) {
-          const int g = w / (rv2 * p.Q);
-          const int rem = w % (rv2 * p.Q);
-          const int q = rem / rv2, m2 = rem % rv2;
-          obuf[(q * G + g) * p.r_v + 2 * m2] = o[vi][0];
-          obuf[(q * G + g) * p.r_v + 2 * m2 + 1] = o[vi][1];
+        for (int e = 0; e < 4; ++e) {
+          obuf[(q * G + g) * p.r_v + 8 * c8 + 2 * e] = o[e].x;
+          obuf[(q * G + g) * p.r_v + 8 * c8 + 2 * e + 1] = o[e].y;
         }
       }
       named_barrier(1, kEpiThreads);
@@ -526,8 +670,7 @@ int env_int(const char* name, int dflt) {
 struct TcPlan {
   bool ok = false;
   int G = 1, nst = 0, nacc = 1, S = 0, tps = 0;
-  TcParams p{};
-  uint32_t smem = 0;
+  size_t ops_bytes = 0;   // workspace for the per-(b, h) operand images
 };
 
 // Shared-memory layout for (D, G, nst); returns total bytes (plus alignment slack).
@@ -545,34 +688,34 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst) {
   uint32_t o = 0;
   p.st_off = o;
   o += nst * p.st_bytes;
+  // two buffers of the query-absorbed B operand and of the bias tile (per item)
   p.b_off = o;
   p.b_head_bytes = D * p.K_pad * 2;
   p.b_sbo = (p.K_pad / 8) * 128;
-  o = al(o + G * p.b_head_bytes, 1024);
+  o = al(o + 2 * G * p.b_head_bytes, 1024);
+  p.bias_head_bytes = D * 16 * 2;
+  p.bias_off = o;
+  o = al(o + 2 * G * p.bias_head_bytes, 1024);
   p.ones_off = o;
   o += 4096;
-  p.bias_off = o;
-  o = al(o + G * D * 16 * 2, 128);
-  p.qc_off = o;
-  o = al(o + G * (D / 2) * 8, 128);
   p.sbuf_off = o;
-  o += G * kTile * 4;
+  o += (kEpiWG - 1) * G * kTile * 4;
   p.p_off = o;
   o += G * kTile * 4;
   p.red_off = o;
   o += G * 4 * 4;
   p.alpha_off = o;
   o = al(o + G * 4, 16);
-  const int rv2 = p.r_v / 2;
-  int Q = kEpiThreads / (G * rv2);
+  const int rv8 = p.r_v / 8;
+  int Q = kEpiThreads / (G * rv8);
   if (Q < 1) Q = 1;
-  if (Q > 8) Q = 8;
+  if (Q > 32) Q = 32;
   p.Q = Q;
-  p.nv_items = G * rv2 * Q;
+  p.nv_items = G * rv8 * Q;
   p.obuf_off = o;
   o = al(o + Q * G * p.r_v * 4, 16);
   p.bar_off = o;
-  o += (2 * nst + 5) * 8;
+  o += (2 * nst + 8) * 8;
   p.misc_off = o;
   o += 16;
   return o + 1024;
@@ -630,6 +773,8 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   }
   pl.tps = (n_tiles + best_s - 1) / best_s;
   pl.S = (n_tiles + pl.tps - 1) / pl.tps;
+  const size_t K_pad = (c.r_k + 15) / 16 * 16;
+  pl.ops_bytes = (size_t)B * c.H * ((size_t)D * K_pad * 2 + (size_t)D * 32);
   pl.ok = true;
   return pl;
 }
@@ -660,14 +805,35 @@ cudaError_t launch_tc_d(int G, const CUtensorMap& mk, const CUtensorMap& mv, con
   }
 }
 
+cudaError_t launch_prep(const DecodeArgs& a, const TcParams& p, cudaStream_t s) {
+  const int chunks = a.d * p.K_pad / 8;
+  dim3 grid((unsigned)a.H, (unsigned)a.B, (unsigned)((chunks + 127) / 128));
+  unsigned char* ob = const_cast<unsigned char*>(p.ops_b);
+  unsigned char* obias = const_cast<unsigned char*>(p.ops_bias);
+#define LLA_PREP(DD)                                                                          \
+  decode_prep_kernel<DD><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, \
+                                              a.muk_t, a.kappa, a.H, a.r_k, p.K_pad, ob, obias, \
+                                              a.status)
+  switch (a.d) {
+    case 32: LLA_PREP(32); break;
+    case 64: LLA_PREP(64); break;
+    case 96: LLA_PREP(96); break;
+    case 128: LLA_PREP(128); break;
+    default: return cudaErrorNotSupported;
+  }
+#undef LLA_PREP
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps) {
+bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps, size_t* ops_bytes) {
   if (!tc_enabled()) return false;
   TcPlan pl = tc_plan(c, B, n_cap);
   if (!pl.ok) return false;
   *S = pl.S;
   *tps = pl.tps;
+  *ops_bytes = pl.ops_bytes;
   return true;
 }
 
@@ -691,21 +857,28 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.HG = a.H / pl.G;
   p.n_items = a.B * p.HG * pl.S;
   p.rope_max_pos = a.rope_max_pos;
-  p.kappa = a.kappa;
   p.nacc = pl.nacc;
   p.acc_cols = pl.G * a.d;
   int cols = 32;
   while (cols < p.nacc * p.acc_cols) cols <<= 1;
   p.tmem_cols = cols;
-  p.wupk_t = a.wupk_t;
-  p.muk_t = a.muk_t;
   p.rope = a.rope;
+  for (int i = 0; i < a.d / 2; ++i) {
+    const double theta = std::pow((double)a.rope_base, -2.0 * i / (double)a.d);
+    const double turns = theta / (2.0 * 3.14159265358979323846);
+    const uint64_t fx = static_cast<uint64_t>(std::ldexp(turns - std::floor(turns), 64));
+    p.phi_lo[i] = static_cast<uint32_t>(fx);
+    p.phi_hi[i] = static_cast<uint32_t>(fx >> 32);
+    const double adv = std::fmod((double)kTile * theta, 2.0 * 3.14159265358979323846);
+    p.step[i] = make_float2((float)std::cos(adv), (float)-std::sin(adv));
+  }
   p.ctx_len = a.ctx_len;
-  p.q = a.q;
   p.positions = a.positions;
-  p.q_pos = a.q_pos;
   p.status = a.status;
   p.partials = a.partials;
+  if (!a.ops) return cudaErrorNotSupported;
+  p.ops_b = a.ops;
+  p.ops_bias = a.ops + (size_t)a.B * a.H * p.b_head_bytes;
   CUtensorMap mk, mv;
   const CUtensorMapSwizzle swz = p.box_k == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -716,6 +889,8 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t pe = launch_prep(a, p, s);
+  if (pe != cudaSuccess) return pe;
   const int grid = p.n_items < sms ? p.n_items : sms;
   switch (a.d) {
     case 32: return launch_tc_d<32>(pl.G, mk, mv, p, smem, grid, s);

@@ -6,7 +6,7 @@
 #include <stdint.h>
 #include <stddef.h>
 
-#include "../../include/lla.h"
+#include "lla.h"
 
 namespace lla {
 
@@ -19,7 +19,8 @@ constexpr int kMaxSplits = 64;      // context splits per (b, h) at most
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Offsets (bytes) of each section of the packed codec buffer.
-//   wup_{k,v}  fp32 [T][H][d][r]      loop-t, head-h up-projection W_up,t,h (d x r)
+//   wup_k      fp32 [T][H][d][r]      loop-t, head-h up-projection W_up,k,t,h (d x r)
+//   wup_v      fp32 [T][H][r][d]      W_up,v,t,h transposed (read column-wise by the combine)
 //   mu_{k,v}   fp32 [T][H][d]         loop-t, head-h mean slice mu_t,h
 //   wd_{k,v}   bf16 [L][r][W]         W_down^T (rows = latent index), L = H (per head) or 1
 //   bias_{k,v} fp32 [L][r]            mu W_down with the bf16-rounded W_down
@@ -37,6 +38,7 @@ struct SplitPlan {
   int splits;           // S
   int tiles_per_split;  // tiles handled by one CTA
   bool tensor_cores;    // the tcgen05 partial kernel takes this shape
+  size_t ops_bytes;     // workspace for its per-(b, h) operand images
 };
 SplitPlan split_plan(const lla_cfg& c, int B, int n_cap);
 size_t partials_bytes(const lla_cfg& c, int B, int S);
@@ -55,8 +57,9 @@ struct DecodeArgs {
   int T, H, d, r_k, r_v, mode;
   float kappa;           // sm_scale * log2(e): scores are kept in base-2 units
   int t, B, n_cap, rope_max_pos;
+  float rope_base;
   const float* wupk_t;   // packed W_up,k at loop t: [H][d][r_k]
-  const float* wupv_t;   // [H][d][r_v]
+  const float* wupv_t;   // [H][r_v][d] (transposed)
   const float* muk_t;    // [H][d]
   const float* muv_t;    // [H][d]
   const float2* rope;    // [rope_max_pos][d/2]
@@ -74,6 +77,7 @@ struct DecodeArgs {
   int32_t* status;       // ws words [0], [1]
   float* partials;       // [B][H][S][2 + r_v]
   int S, tiles_per_split;
+  unsigned char* ops;    // per-(b, h) MMA operand images (tensor-core path), or null
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
@@ -81,7 +85,7 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 // Tensor-core (tcgen05) partial kernel for per-head decode.  decode_tc_plan
 // reports whether the shape takes that path and its context split; the launcher
 // returns cudaErrorNotSupported when it cannot run the shape.
-bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps);
+bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps, size_t* ops_bytes);
 cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t s);
 
 // Record `fmt` as the calling thread's lla_last_error() message; returns `code`.

@@ -68,19 +68,30 @@ __global__ void rope_table_kernel(int max_pos, int half, double base, float2* ta
 
 // ---------------------------------------------------------------- packing
 
-// W_up: per head [H][T][d][r] -> [T][H][d][r]; LLA-2D input is already [T][H][d][r].
+// W_up: per head [H][T][d][r] (LLA-2D [T][H][d][r]) -> [T][H][d][r], or with
+// transpose != 0 -> [T][H][r][d] (the V up-projection, read column-wise).
 __global__ void pack_wup_kernel(const float* __restrict__ in, float* __restrict__ out, int T,
-                                int H, int d, int r, int per_head) {
+                                int H, int d, int r, int per_head, int transpose) {
   const long long n = (long long)T * H * d * r;
   for (long long o = (long long)blockIdx.x * blockDim.x + threadIdx.x; o < n;
        o += (long long)gridDim.x * blockDim.x) {
-    const int m = (int)(o % r);
-    long long rest = o / r;
-    const int i = (int)(rest % d);
-    rest /= d;
+    int m, i;
+    long long rest;
+    if (transpose) {
+      i = (int)(o % d);
+      rest = o / d;
+      m = (int)(rest % r);
+      rest /= r;
+    } else {
+      m = (int)(o % r);
+      rest = o / r;
+      i = (int)(rest % d);
+      rest /= d;
+    }
     const int h = (int)(rest % H);
     const int t = (int)(rest / H);
-    const long long src = per_head ? ((((long long)h * T + t) * d + i) * r + m) : o;
+    const long long src = per_head ? ((((long long)h * T + t) * d + i) * r + m)
+                                   : ((((long long)t * H + h) * d + i) * r + m);
     out[o] = in[src];
   }
 }
@@ -344,48 +355,71 @@ __global__ void __launch_bounds__(128) decode_partial_kernel(DecodeArgs a) {
   }
 }
 
-// Merge the splits, add the in-flight token and up-project V once.  One CTA per (h, b).
-__global__ void __launch_bounds__(128) decode_combine_kernel(DecodeArgs a) {
-  __shared__ float olat[256];
-  __shared__ float red[8];
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const size_t bh = (size_t)b * a.H + h;
-  const float* qh = a.q + bh * a.d;
-  const float* kh = a.k_self + bh * a.d;
-  // Same position for query and key: the relative rotation is the identity.
-  float part_dot = 0.f;
-  for (int i = tid; i < a.d; i += blockDim.x) part_dot = fmaf(qh[i], kh[i], part_dot);
-  const float s_self = a.kappa * block_sum128(part_dot, red);
+// Merge the splits, add the in-flight token and up-project V once.
+// Grid (H, B, ceil(d / 32)); 512 threads.  Block z computes output rows
+// [32 z, 32 z + 32) of (b, h); every phase issues all of its global loads at once.
+constexpr int kCombineThreads = 512;
 
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(DecodeArgs a) {
+  __shared__ float olat[256];
+  __shared__ float mw[kMaxSplits];
+  __shared__ float red[16];
+  __shared__ float seg[16][33];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const size_t bh = (size_t)b * a.H + h;
   const float* parts = a.partials + bh * a.S * (2 + a.r_v);
-  float M = s_self;
-  for (int s = 0; s < a.S; ++s) M = fmaxf(M, parts[(size_t)s * (2 + a.r_v)]);
-  const float w_self = exp2f(s_self - M);
-  float l_hist = 0.f;
-  for (int s = 0; s < a.S; ++s) {
-    const float* ps = parts + (size_t)s * (2 + a.r_v);
-    l_hist += ps[1] * exp2f(ps[0] - M);
+  // split maxima, and the in-flight token's score
+  // (same position for query and key: their relative rotation is the identity)
+  float m_s = -INFINITY, dot = 0.f;
+  if (tid < a.S) m_s = parts[(size_t)tid * (2 + a.r_v)];
+  if (tid < a.d) dot = a.q[bh * a.d + tid] * a.k_self[bh * a.d + tid];
+  const float mx = warp_max(m_s), dsum = warp_sum(dot);
+  if (lane == 0) {
+    red[warp] = mx;
+    seg[warp][32] = dsum;
   }
+  __syncthreads();
+  float M_hist = red[0], s_self = 0.f;
+  for (int w = 1; w < 16; ++w) M_hist = fmaxf(M_hist, red[w]);
+  for (int w = 0; w < 16; ++w) s_self += seg[w][32];
+  s_self *= a.kappa;
+  const float M = fmaxf(M_hist, s_self);
+  const float wgt = tid < a.S ? exp2f(m_s - M) : 0.f;
+  if (tid < a.S) mw[tid] = wgt;
+  __syncthreads();
+  float l_hist = 0.f;
+  for (int s = 0; s < a.S; ++s) l_hist = fmaf(parts[(size_t)s * (2 + a.r_v) + 1], mw[s], l_hist);
+  const float w_self = exp2f(s_self - M);
   const float inv = 1.f / (l_hist + w_self);
-  for (int m = tid; m < a.r_v; m += blockDim.x) {
+  for (int m = tid; m < a.r_v; m += kCombineThreads) {
     float acc = 0.f;
-    for (int s = 0; s < a.S; ++s) {
-      const float* ps = parts + (size_t)s * (2 + a.r_v);
-      acc = fmaf(ps[2 + m], exp2f(ps[0] - M), acc);
-    }
+    for (int s = 0; s < a.S; ++s) acc = fmaf(parts[(size_t)s * (2 + a.r_v) + 2 + m], mw[s], acc);
     olat[m] = acc * inv;
   }
   __syncthreads();
-  const float* Wv = a.wupv_t + (size_t)h * a.d * a.r_v;  // [d][r_v]
-  const float* muv = a.muv_t + (size_t)h * a.d;
-  const float* vs = a.v_self + bh * a.d;
-  for (int i = tid; i < a.d; i += blockDim.x) {
-    const float* row = Wv + (size_t)i * a.r_v;
-    float acc = 0.f;
-    for (int m = 0; m < a.r_v; ++m) acc = fmaf(row[m], olat[m], acc);
-    a.out[bh * a.d + i] = acc + (l_hist * inv) * muv[i] + (w_self * inv) * vs[i];
+  // W_up,v,t,h is packed transposed ([r_v][d]); warp w sums latent dims m = w, w + 16, ...
+  // for the 32 rows i of this block (lane = row), all loads independent.
+  const int i = blockIdx.z * 32 + lane;
+  const float* Wt = a.wupv_t + (size_t)h * a.d * a.r_v;
+  float acc = 0.f;
+  if (i < a.d) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int m = warp + 16 * k;
+      if (m < a.r_v) acc = fmaf(Wt[(size_t)m * a.d + i], olat[m], acc);
+    }
   }
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
+  seg[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0 && i < a.d) {
+    float y = 0.f;
+#pragma unroll
+    for (int w = 0; w < 16; ++w) y += seg[w][lane];
+    const float* muv = a.muv_t + (size_t)h * a.d;
+    a.out[bh * a.d + i] = y + (l_hist * inv) * muv[i] + (w_self * inv) * a.v_self[bh * a.d + i];
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0) {
     a.status[1] = a.status[0];
     a.status[0] = 0;
   }
@@ -414,9 +448,9 @@ cudaError_t launch_pack(const lla_cfg& c, const PackedLayout& L, const float* wd
   const int per_head = c.mode == LLA_MODE_PER_HEAD;
   const int T = c.T, H = c.H, d = c.d_head;
   pack_wup_kernel<<<512, 256, 0, s>>>(wupk, reinterpret_cast<float*>(packed + L.wupk), T, H, d,
-                                      c.r_k, per_head);
+                                      c.r_k, per_head, 0);
   pack_wup_kernel<<<512, 256, 0, s>>>(wupv, reinterpret_cast<float*>(packed + L.wupv), T, H, d,
-                                      c.r_v, per_head);
+                                      c.r_v, per_head, 1);
   pack_mu_kernel<<<64, 256, 0, s>>>(muk, reinterpret_cast<float*>(packed + L.muk), T, H, d, per_head);
   pack_mu_kernel<<<64, 256, 0, s>>>(muv, reinterpret_cast<float*>(packed + L.muv), T, H, d, per_head);
   auto* wdk_bf = reinterpret_cast<__nv_bfloat16*>(packed + L.wdk);
@@ -469,8 +503,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches) {
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
-  dim3 g2((unsigned)a.H, (unsigned)a.B);
-  decode_combine_kernel<<<g2, 128, 0, s>>>(a);
+  dim3 g2((unsigned)a.H, (unsigned)a.B, (unsigned)((a.d + 31) / 32));
+  decode_combine_kernel<<<g2, kCombineThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
