@@ -41,17 +41,23 @@ using namespace sm100;
 constexpr int kEpiWG = 2;                       // epilogue warpgroups
 constexpr int kEpiThreads = 128 * kEpiWG;       // warps 2 .. 2 + 4 kEpiWG - 1
 constexpr int kEpiWarps = kEpiThreads / 32;
-constexpr int kThreads = 64 + kEpiThreads;      // warp 0 TMA, warp 1 MMA, then the epilogue
+// warp 0: c_k producer, warp 1: score MMA issuer, warps 2..9: epilogue,
+// warp 10: c_v producer, warp 11: V MMA issuer
+constexpr int kThreads = 64 + kEpiThreads + 64;
+constexpr int kVProdWarp = 2 + kEpiWarps, kVMmaWarp = 3 + kEpiWarps;
 constexpr uint32_t kSmemLimit = 232448;  // per-block dynamic shared memory on sm_100
 
 struct TcParams {
-  int H, r_k, r_v, K_pad, box_k, nkb, swz;   // swz: descriptor swizzle code
-  int Q, nv_items;                           // V-phase split: token residues, work items
+  int H, r_k, r_v, K_pad, box_k, nkb, swz;   // K latent tiles: K-major, swizzle code swz
+  int nst_v;                                 // V latent ring depth (nst: K latent ring)
+  uint32_t stv_off, stv_bytes, tx_v;
+  int N_v, cvb, nvb, swz_v;                  // V latent tiles: MN-major boxes of cvb dims
+  int nmb;                                   // 128-dim blocks of the V latent (V MMA rows)
   int B, n_cap, S, tps, HG, n_items, rope_max_pos;
-  uint32_t st_off, st_bytes, cv_off, box_bytes;
+  uint32_t st_off, st_bytes, cv_off, box_bytes, vbox_bytes;
   uint32_t b_off, b_head_bytes, b_sbo, bias_head_bytes, ones_off, bias_off, sbuf_off, p_off,
-      red_off, alpha_off, obuf_off, bar_off, misc_off;
-  int nst, nacc, acc_cols, tmem_cols;
+      red_off, ctx_off, rope_off, bar_off, misc_off;
+  int nst, nacc, acc_cols, v_col0, tmem_cols;
   uint32_t tx_bytes;
   const float2* rope;    // [rope_max_pos][d/2]
   const int32_t* ctx_len;
@@ -118,6 +124,37 @@ __device__ __forceinline__ int epi_barrier_or(int pred) {
   return static_cast<int>(out);
 }
 
+// registers -> TMEM, 16 consecutive columns (32x32b shape).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float* v) {
+  uint32_t r0, r1;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
+  v[0] = __uint_as_float(r0);
+  v[1] = __uint_as_float(r1);
+}
+
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, float v0, float v1) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr),
+               "r"(__float_as_uint(v0)), "r"(__float_as_uint(v1))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // TMEM -> registers, 8 consecutive columns (32x32b shape).
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
   uint32_t r[8];
@@ -134,16 +171,25 @@ struct ItemRange {
   int b, hg, s, tok0, tok_end, ntiles;
 };
 
-__device__ __forceinline__ ItemRange item_range(const TcParams& p, int item, bool flag_ctx) {
+constexpr int kCtxCache = 1024;   // sequences whose context length is cached in smem
+
+// ctx_s: clamped context lengths cached in shared memory (B <= kCtxCache), else null.
+__device__ __forceinline__ ItemRange item_range(const TcParams& p, const int* ctx_s, int item,
+                                                bool flag_ctx) {
   ItemRange r;
   r.s = item % p.S;
   const int u = item / p.S;
   r.hg = u % p.HG;
   r.b = u / p.HG;
-  int n = p.ctx_len[r.b];
-  if (n < 0 || n > p.n_cap) {
-    if (flag_ctx) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
-    n = n < 0 ? 0 : p.n_cap;
+  int n;
+  if (ctx_s) {
+    n = ctx_s[r.b];
+  } else {
+    n = p.ctx_len[r.b];
+    if (n < 0 || n > p.n_cap) {
+      if (flag_ctx) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
+      n = n < 0 ? 0 : p.n_cap;
+    }
   }
   r.tok0 = r.s * p.tps * kTile;
   r.tok_end = min(r.tok0 + p.tps * kTile, n);
@@ -158,11 +204,11 @@ struct TileCursor {
   bool valid;
 };
 
-__device__ __forceinline__ void cursor_first(const TcParams& p, TileCursor& c) {
+__device__ __forceinline__ void cursor_first(const TcParams& p, const int* ctx_s, TileCursor& c) {
   c.valid = false;
   c.k = 0;
   for (c.item = blockIdx.x; c.item < p.n_items; c.item += gridDim.x) {
-    c.r = item_range(p, c.item, false);
+    c.r = item_range(p, ctx_s, c.item, false);
     if (c.r.ntiles > 0) {
       c.valid = true;
       return;
@@ -170,12 +216,12 @@ __device__ __forceinline__ void cursor_first(const TcParams& p, TileCursor& c) {
   }
 }
 
-__device__ __forceinline__ void cursor_next(const TcParams& p, TileCursor& c) {
+__device__ __forceinline__ void cursor_next(const TcParams& p, const int* ctx_s, TileCursor& c) {
   if (!c.valid) return;
   if (++c.k < c.r.ntiles) return;
   c.k = 0;
   for (c.item += gridDim.x; c.item < p.n_items; c.item += gridDim.x) {
-    c.r = item_range(p, c.item, false);
+    c.r = item_range(p, ctx_s, c.item, false);
     if (c.r.ntiles > 0) return;
   }
   c.valid = false;
@@ -267,6 +313,10 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
   }
 }
 
+// log2 of the largest softmax weight a tile may carry before the V accumulator
+// is rescaled to a new reference maximum.
+constexpr float kRescaleLog2 = 8.f;
+
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap map_k,
@@ -277,28 +327,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + p.bar_off);
-  uint64_t* empty = full + p.nst;
-  uint64_t* tfull = empty + p.nst;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* bfull = tempty + 2;    // [2] B operand buffers loaded
-  uint64_t* bempty = bfull + 2;    // [2] B operand buffers free (MMAs done)
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(sm + p.bar_off);   // [nst] K latent tile landed
+  uint64_t* empty_k = full_k + p.nst;                                // [nst] score MMA done with it
+  uint64_t* full_v = empty_k + p.nst;                                // [nst_v] V latent tile landed
+  uint64_t* empty_v = full_v + p.nst_v;                              // [nst_v] V MMA done with it
+  uint64_t* tfull = empty_v + p.nst_v;   // [2] scores in TMEM
+  uint64_t* tempty = tfull + 2;          // [2] scores read
+  uint64_t* bfull = tempty + 2;          // [2] query-absorbed operands loaded
+  uint64_t* bempty = bfull + 2;          // [2] operand buffer free
+  uint64_t* pfull = bempty + 2;          // [2] softmax weights written
+  uint64_t* pempty = pfull + 2;          // [2] V MMA done with the weights buffer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t ops_head_bytes = p.b_head_bytes;
+  const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.nst; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kEpiWarps);
+      mbar_init(&full_k[s], 1);
+      mbar_init(&empty_k[s], 1);
+    }
+    for (int s = 0; s < p.nst_v; ++s) {
+      mbar_init(&full_v[s], 1);
+      mbar_init(&empty_v[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kEpiWarps);
       mbar_init(&bfull[a], 1);
       mbar_init(&bempty[a], 1);
+      mbar_init(&pfull[a], 1);
+      mbar_init(&pempty[a], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -307,14 +368,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, p.tmem_cols);
     tmem_relinquish();
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 2 + kEpiWarps) {
     const int et = threadIdx.x - 64;
-    // ones tile [128 x 16]: columns 0 and 1 hold 1.0 (adds bias hi + lo to every row).
-    for (int idx = et; idx < 128 * 16; idx += kEpiThreads) {
-      const int m = idx / 16, k = idx % 16;
-      const uint32_t off = p.ones_off + (m >> 3) * 256 + (k >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2;
-      *reinterpret_cast<__nv_bfloat16*>(sm + off) = __float2bfloat16_rn(k < 2 ? 1.f : 0.f);
+    if (ctx_s) {
+      int* cs = reinterpret_cast<int*>(sm + p.ctx_off);
+      for (int b = et; b < p.B; b += kEpiThreads) {
+        int n = p.ctx_len[b];
+        if (n < 0 || n > p.n_cap) {
+          if (blockIdx.x == 0) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
+          n = n < 0 ? 0 : p.n_cap;
+        }
+        cs[b] = n;
+      }
     }
+    if (et < 64) {
+      reinterpret_cast<float2*>(sm + p.rope_off)[et] = p.step[et];
+      reinterpret_cast<uint2*>(sm + p.rope_off + 512)[et] = make_uint2(p.phi_lo[et], p.phi_hi[et]);
+    }
+    // ones tile: one 8-row group (K columns 0 and 1 hold 1.0) that every row group aliases
+    if (et < 8 * 16) {
+      const int m = et / 16, k = et % 16;
+      *reinterpret_cast<__nv_bfloat16*>(sm + p.ones_off + (k >> 3) * 128 + m * 16 + (k & 7) * 2) =
+          __float2bfloat16_rn(k < 2 ? 1.f : 0.f);
+    }
+    // softmax-weight tiles (two buffers x G heads, 8 rows x 128 tokens): rows 2..7 stay 0
+    for (int idx = et; idx < 2 * G * 8 * kTile / 2; idx += kEpiThreads)
+      reinterpret_cast<uint32_t*>(sm + p.p_off)[idx] = 0u;
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -322,17 +401,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == kVProdWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0 streams the K latents (and each item's operand images), warp kVProdWarp
+    // the V latents; each ring is released by the MMA that reads it.
     if (lane == 0) {
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
+      const bool kside = warp == 0;
+      const CUtensorMap* map = kside ? &map_k : &map_v;
+      tma_prefetch_desc(map);
+      const int nst = kside ? p.nst : p.nst_v;
+      uint64_t* fullb = kside ? full_k : full_v;
+      uint64_t* emptyb = kside ? empty_k : empty_v;
       uint32_t it = 0, jn = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const ItemRange r = item_range(p, item, false);
+        const ItemRange r = item_range(p, ctx_s, item, false);
         if (r.ntiles == 0) continue;
-        {
+        if (kside) {
           // query-absorbed operands of this item into B buffer jn & 1
           const uint32_t buf = jn & 1u, bph = (jn >> 1) & 1u;
           if (!mbar_wait(&bempty[buf], bph ^ 1u, abort_flag)) break;
@@ -345,36 +430,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++jn;
         }
         for (int k = 0; k < r.ntiles; ++k, ++it) {
-          const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
-          if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) {
+          const uint32_t stage = it % nst, ph = (it / nst) & 1u;
+          if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], p.tx_bytes);
-          unsigned char* st = sm + p.st_off + stage * p.st_bytes;
           const int y = r.tok0 + k * kTile;
+          if (kside) {
+            mbar_arrive_expect_tx(&fullb[stage], p.tx_bytes);
+            unsigned char* st = sm + p.st_off + stage * p.st_bytes;
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const int h = r.hg * G + g;
-            for (int kb = 0; kb < p.nkb; ++kb)
-              tma_load_3d(st + (g * p.nkb + kb) * p.box_bytes, &map_k, &full[stage],
-                          h * p.r_k + kb * p.box_k, y, r.b);
-            tma_load_3d(st + p.cv_off + g * (kTile * p.r_v * 2), &map_v, &full[stage], h * p.r_v,
-                        y, r.b);
+            for (int g = 0; g < G; ++g) {
+              const int h = r.hg * G + g;
+              for (int kb = 0; kb < p.nkb; ++kb)
+                tma_load_3d(st + (g * p.nkb + kb) * p.box_bytes, map, &fullb[stage],
+                            h * p.r_k + kb * p.box_k, y, r.b);
+            }
+          } else {
+            mbar_arrive_expect_tx(&fullb[stage], p.tx_v);
+            unsigned char* st = sm + p.stv_off + stage * p.stv_bytes;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const int h = r.hg * G + g;
+              for (int vb = 0; vb < p.nvb; ++vb)
+                tma_load_3d(st + (g * p.nvb + vb) * p.vbox_bytes, map, &fullb[stage],
+                            h * p.r_v + vb * p.cvb, y, r.b);
+            }
           }
         }
       }
       if (*abort_flag) {
         // Drain: wait (bounded) for every copy this thread issued before leaving.
-        const uint32_t n_out = it < (uint32_t)p.nst ? it : (uint32_t)p.nst;
+        const uint32_t n_out = it < (uint32_t)nst ? it : (uint32_t)nst;
         for (uint32_t j = 0; j < n_out; ++j) {
           const uint32_t i = it - 1 - j;
-          const uint32_t stage = i % p.nst, ph = (i / p.nst) & 1u;
+          const uint32_t stage = i % nst, ph = (i / nst) & 1u;
           const unsigned long long t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[stage], ph) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+          while (!mbar_try_wait(&fullb[stage], ph) && global_timer_ns() - t0 < kWaitTimeoutNs) {
           }
         }
-        for (uint32_t j = 0; j < 2 && j < jn; ++j) {
+        for (uint32_t j = 0; kside && j < 2 && j < jn; ++j) {
           const uint32_t i = jn - 1 - j;
           const unsigned long long t0 = global_timer_ns();
           while (!mbar_try_wait(&bfull[i & 1u], (i >> 1) & 1u) &&
@@ -384,25 +479,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D);
       const uint32_t sbo_a = 16u * p.box_k;
-      const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 256, 0);
+      const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 0, 0);   // rows alias
       uint32_t it = 0, jn = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const ItemRange r = item_range(p, item, false);
+        const ItemRange r = item_range(p, ctx_s, item, false);
         if (r.ntiles == 0) continue;
         const uint32_t buf = jn & 1u, bph = (jn >> 1) & 1u;
-        if (!mbar_wait(&bfull[buf], bph, abort_flag)) break;
+        if (!mbar_wait(&bfull[buf], bph, abort_flag)) {
+          ok = false;
+          break;
+        }
         ++jn;
         const uint32_t b_base = smem_addr(sm + p.b_off + buf * G * ops_head_bytes);
         const uint32_t bias_base = smem_addr(sm + p.bias_off + buf * G * p.bias_head_bytes);
         for (int k = 0; k < r.ntiles; ++k, ++it) {
           const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
           const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
-          if (!mbar_wait(&full[stage], ph, abort_flag) ||
+          if (!mbar_wait(&full_k[stage], ph, abort_flag) ||
               !mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -424,50 +522,89 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16(d_tmem, odesc, bias_desc, idesc, 1u);
           }
           mma_commit(&tfull[acc]);
+          mma_commit(&empty_k[stage]);
+          if (k == r.ntiles - 1) mma_commit(&bempty[buf]);   // last use of this B buffer
         }
-        if (ok) mma_commit(&bempty[buf]);   // B buffer reusable once these MMAs finish
+      }
+    }
+    __syncwarp();
+  } else if (warp == kVMmaWarp) {
+    // ------------------------------------------------------------ V MMA issuer
+    // D_v[g] (+)= P_i[g] (rows 0, 1: weights hi, lo; all 8-row groups alias) x C_v,i[g]
+    // (128 tokens x N_v latent dims, MN-major): one K=16 MMA per 16 tokens.
+    if (lane == 0) {
+      const uint32_t idesc_v = idesc_bf16_f32(128, p.N_v) | (1u << 16);   // B (c_v) MN-major
+      const uint32_t sbo_v = 16u * p.cvb;          // 8 token rows of one MN box
+      const uint32_t p_base = smem_addr(sm + p.p_off);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t pb = it & 1u;
+          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag) ||
+              !mbar_wait(&full_v[vs], vph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t cv_addr = smem_addr(sm + p.stv_off + vs * p.stv_bytes);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint32_t d_tmem = tmem_base + p.v_col0 + g * p.N_v;
+            const uint32_t a_addr = p_base + (pb * G + g) * (8 * kTile * 2);
+            const uint32_t b_addr = cv_addr + g * p.nvb * p.vbox_bytes;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t adesc = smem_desc(a_addr + kk * 256, 128, 0, 0);
+              const uint64_t bdesc =
+                  smem_desc(b_addr + kk * 2 * sbo_v, p.vbox_bytes, sbo_v, p.swz_v);
+              mma_bf16(d_tmem, adesc, bdesc, idesc_v, (k == 0 && kk == 0) ? 0u : 1u);
+            }
+          }
+          mma_commit(&pempty[pb]);
+          mma_commit(&empty_v[vs]);
+        }
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;
-    const int wgi = (warp - 2) >> 2;          // which quarter of the RoPE pairs
+    const int wgi = (warp - 2) >> 2;          // which part of the RoPE pairs
     const int sub = warp & 3;                 // TMEM sub-partition of this warp
     const int row = sub * 32 + lane;          // token row of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
-    float* sbuf = reinterpret_cast<float*>(sm + p.sbuf_off);   // [kEpiWG - 1][G][128]
-    float* P = reinterpret_cast<float*>(sm + p.p_off);         // [G][128]
+    float* sbuf = reinterpret_cast<float*>(sm + p.sbuf_off);   // [2][kEpiWG - 1][G][128]
     float* red = reinterpret_cast<float*>(sm + p.red_off);     // [G][4]
-    float* alpha_s = reinterpret_cast<float*>(sm + p.alpha_off);
-    float* obuf = reinterpret_cast<float*>(sm + p.obuf_off);   // [Q][G][r_v]
-    const int rv8 = p.r_v >> 3;
 
-    // Software pipeline of the RoPE factors: the table row of tile it+1 is loaded
-    // while tile it is processed, and positions two tiles ahead.
     TileCursor pc;
-    cursor_first(p, pc);
+    cursor_first(p, ctx_s, pc);
     // conj(e^{i p theta_i}) for this thread's RoPE pairs at position pos_cur of its
     // token; when the next tile's token sits exactly one tile further on, the
     // factors advance by one complex product, otherwise they are recomputed.
     float2 ef[WG_PAIRS];
     int pos_cur = kNoPos, run = 0;
+    const float2* step_s = reinterpret_cast<const float2*>(sm + p.rope_off) + wgi * WG_PAIRS;
+    const uint2* phi_s = reinterpret_cast<const uint2*>(sm + p.rope_off + 512) + wgi * WG_PAIRS;
     auto advance_rope = [&](int praw) {
       if (praw == kNoPos) return;               // row past the context: keep factors
       const int pn = checked_pos(p, praw);
       if (pos_cur != kNoPos && pn == pos_cur + kTile && run < kReseedTiles) {
 #pragma unroll
         for (int q = 0; q < WG_PAIRS; ++q) {
-          const float2 st = p.step[wgi * WG_PAIRS + q];
+          const float2 st = step_s[q];
           const float2 e = ef[q];
           ef[q] = make_float2(fmaf(e.x, st.x, -e.y * st.y), fmaf(e.x, st.y, e.y * st.x));
         }
         ++run;
       } else {
 #pragma unroll
-        for (int q = 0; q < WG_PAIRS; ++q)
-          ef[q] = rope_factor(static_cast<uint32_t>(pn), p.phi_lo[wgi * WG_PAIRS + q],
-                              p.phi_hi[wgi * WG_PAIRS + q]);
+        for (int q = 0; q < WG_PAIRS; ++q) {
+          const uint2 ph = phi_s[q];
+          ef[q] = rope_factor(static_cast<uint32_t>(pn), ph.x, ph.y);
+        }
         run = 0;
       }
       pos_cur = pn;
@@ -475,24 +612,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int q = 0; q < WG_PAIRS; ++q) ef[q] = make_float2(1.f, 0.f);
     advance_rope(cursor_pos(p, pc, row));
-    cursor_next(p, pc);
+    cursor_next(p, ctx_s, pc);
     int pos_next = cursor_pos(p, pc, row);
-    cursor_next(p, pc);
+    cursor_next(p, ctx_s, pc);
 
     uint32_t it = 0;
     bool aborted = false;
     for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
-      const ItemRange r = item_range(p, item, et == 0);
-      float m_run[G], l_part[G];
+      const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
+      float m_ref[G], l_part[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        m_run[g] = -INFINITY;
+        m_ref[g] = -INFINITY;
         l_part[g] = 0.f;
       }
-      float2 o[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                     make_float2(0.f, 0.f)};
       for (int k = 0; k < r.ntiles; ++k, ++it) {
-        const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
         const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
         const int t0 = r.tok0 + k * kTile;
         const int cnt = min(kTile, r.tok_end - t0);
@@ -503,122 +637,152 @@ __global__ void __launch_bounds__(kThreads, 1)
         float part[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          part[g] = 0.f;
           const uint32_t col = tmem_base + lane_addr + acc * p.acc_cols + g * D + wgi * WG_COLS;
           float u[WG_COLS];
 #pragma unroll
           for (int c = 0; c < WG_COLS / 16; ++c) tmem_ld16(col + c * 16, u + c * 16);
           if constexpr (WG_COLS % 16 != 0) tmem_ld8(col + (WG_COLS / 16) * 16, u + (WG_COLS / 16) * 16);
           tmem_wait_ld();
-          float2 acc2 = make_float2(0.f, 0.f);
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int q = 0; q < WG_PAIRS; ++q) acc2 = ffma2(make_float2(u[2 * q], u[2 * q + 1]), ef[q], acc2);
-          part[g] = acc2.x + acc2.y;
+          for (int q = 0; q < WG_PAIRS; q += 2) {
+            a0 = ffma2(make_float2(u[2 * q], u[2 * q + 1]), ef[q], a0);
+            if (q + 1 < WG_PAIRS) a1 = ffma2(make_float2(u[2 * q + 2], u[2 * q + 3]), ef[q + 1], a1);
+          }
+          part[g] = (a0.x + a0.y) + (a1.x + a1.y);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
-        // RoPE factors of the next tile (its position was loaded a tile ago), and
-        // the raw position of the tile after it
-        advance_rope(pos_next);
-        pos_next = cursor_pos(p, pc, row);
-        cursor_next(p, pc);
-        ok = ok && mbar_wait(&full[stage], ph, abort_flag);
         if (wgi > 0) {
 #pragma unroll
-          for (int g = 0; g < G; ++g) sbuf[((wgi - 1) * G + g) * kTile + row] = part[g];
+          for (int g = 0; g < G; ++g)
+            sbuf[(((it & 1u) * (kEpiWG - 1) + (wgi - 1)) * G + g) * kTile + row] = part[g];
         }
         if (epi_barrier_or(!ok)) {
           aborted = true;
           break;
         }
         if (wgi == 0) {
+          // ---- softmax weights against the item's reference maximum m_ref
           float s[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             float tot = part[g];
 #pragma unroll
-            for (int w = 0; w < kEpiWG - 1; ++w) tot += sbuf[(w * G + g) * kTile + row];
+            for (int w = 0; w < kEpiWG - 1; ++w)
+              tot += sbuf[(((it & 1u) * (kEpiWG - 1) + w) * G + g) * kTile + row];
             s[g] = valid ? tot : -INFINITY;
             const float mx = warp_max_f(s[g]);
             if (lane == 0) red[g * 4 + sub] = mx;
           }
           named_barrier(2, 128);
+          bool rescale = false;
+          float alpha[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float mt = fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
-            const float m_new = fmaxf(m_run[g], mt);
-            const float alpha = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - m_new);
-            const float pj = valid ? exp2f(s[g] - m_new) : 0.f;
-            P[g * kTile + row] = pj;
-            l_part[g] = l_part[g] * alpha + pj;
-            m_run[g] = m_new;
-            if (row == 0) alpha_s[g] = alpha;
+            alpha[g] = 1.f;
+            if (k == 0) {
+              m_ref[g] = mt;
+            } else if (mt > m_ref[g] + kRescaleLog2) {
+              alpha[g] = exp2f(m_ref[g] - mt);
+              m_ref[g] = mt;
+              rescale = true;
+            }
           }
-        }
-        named_barrier(1, kEpiThreads);
-        // latent-space V accumulation from the staged c_v tile: thread = (head,
-        // 8 latent dims, token residue q); tokens j = q, q + Q, ...
-        if (et < p.nv_items) {
-          const unsigned char* cvb = sm + p.st_off + stage * p.st_bytes + p.cv_off;
-          const int g = et / (rv8 * p.Q);
-          const int rem = et % (rv8 * p.Q);
-          const int q = rem / rv8, c8 = rem % rv8;
-          const float a = alpha_s[g];
+          const uint32_t pb = it & 1u;
+          // the weights buffer is free once the V MMA of tile it - 2 has finished
+          ok = mbar_wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u, abort_flag);
+          if (rescale) {
+            // rare: rescale the item's V accumulator (TMEM lanes 0 and 1) once the V MMA
+            // of the previous tile has finished; sub-partition 0 (lanes 0-31) does it
+            ok = ok && mbar_wait(&pempty[(it - 1) & 1u], ((it - 1) >> 1) & 1u, abort_flag);
+            tc_fence_after();
+            if (sub == 0) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[e] = make_float2(o[e].x * a, o[e].y * a);
-          const uint4* cv = reinterpret_cast<const uint4*>(cvb + g * (kTile * p.r_v * 2)) + c8;
-          const float* Pg = P + g * kTile;
-#pragma unroll 2
-          for (int j = q; j < cnt; j += p.Q) {
-            const float pj = Pg[j];
-            const float2 pj2 = make_float2(pj, pj);
-            const uint4 raw = cv[(size_t)j * rv8];
-            const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+              for (int g = 0; g < G; ++g) {
+                for (int c = 0; c < p.N_v; c += 16) {
+                  float v[16];
+                  const uint32_t ta = tmem_base + p.v_col0 + g * p.N_v + c;
+                  tmem_ld16(ta, v);
+                  tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[e] = ffma2(pj2, __bfloat1622float2(v2[e]), o[e]);
+                  for (int e = 0; e < 16; ++e) v[e] *= alpha[g];
+                  tmem_st16(ta, v);
+                }
+              }
+              tmem_wait_st();
+            }
+            tc_fence_before();
           }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float pj = valid ? exp2f(s[g] - m_ref[g]) : 0.f;
+            l_part[g] = l_part[g] * alpha[g] + pj;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(pj);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(pj - __bfloat162float(hi));
+            unsigned char* pt = sm + p.p_off + (pb * G + g) * (8 * kTile * 2) +
+                                (row >> 3) * 128 + (row & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(pt) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(pt + 16) = lo;
+          }
+          fence_proxy_async_smem();
+          named_barrier(2, 128);
+          if (row == 0) mbar_arrive(&pfull[pb]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (!ok) *abort_flag = 1;
+        // off the critical path: RoPE factors of the next tile (its position was
+        // loaded a tile ago) and the raw position of the tile after it
+        advance_rope(pos_next);
+        pos_next = cursor_pos(p, pc, row);
+        cursor_next(p, ctx_s, pc);
       }
       if (aborted) break;
       // ---------------------------------------------------------- item partial
-      const size_t bh0 = (size_t)r.b * p.H + r.hg * G;
-      if (wgi == 0) {
+      if (wgi == 0 && r.ntiles > 0) {
+        const size_t bh0 = (size_t)r.b * p.H + r.hg * G;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float l = warp_sum_f(l_part[g]);
           if (lane == 0) red[g * 4 + sub] = l;
         }
+        // V accumulator: wait for the item's last V MMA, then read lanes 0 (hi) and 1 (lo)
+        const uint32_t last = it - 1;
+        const bool okv =
+            __all_sync(0xffffffffu, mbar_wait(&pempty[last & 1u], (last >> 1) & 1u, abort_flag));
+        tc_fence_after();
         named_barrier(2, 128);
-        if (row == 0) {
+        if (sub == 0 && okv) {
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             float* part_out = p.partials + ((bh0 + g) * p.S + r.s) * (2 + p.r_v);
-            part_out[0] = m_run[g];
-            part_out[1] = red[g * 4] + red[g * 4 + 1] + red[g * 4 + 2] + red[g * 4 + 3];
+            if (lane == 0) {
+              part_out[0] = m_ref[g];
+              part_out[1] = red[g * 4] + red[g * 4 + 1] + red[g * 4 + 2] + red[g * 4 + 3];
+            }
+            for (int c = 0; c < p.N_v; c += 16) {
+              float v[16];
+              tmem_ld16(tmem_base + p.v_col0 + g * p.N_v + c, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float o = v[e] + __shfl_down_sync(0xffffffffu, v[e], 1);
+                if (lane == 0 && c + e < p.r_v) part_out[2 + c + e] = o;
+              }
+            }
           }
         }
-      }
-      if (et < p.nv_items) {
-        const int g = et / (rv8 * p.Q);
-        const int rem = et % (rv8 * p.Q);
-        const int q = rem / rv8, c8 = rem % rv8;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          obuf[(q * G + g) * p.r_v + 8 * c8 + 2 * e] = o[e].x;
-          obuf[(q * G + g) * p.r_v + 8 * c8 + 2 * e + 1] = o[e].y;
+        tc_fence_before();
+        named_barrier(2, 128);
+      } else if (wgi == 0) {
+        // no tiles in this split: empty partial
+        const size_t bh0 = (size_t)r.b * p.H + r.hg * G;
+        for (int idx = row; idx < G * (2 + p.r_v); idx += 128) {
+          const int g = idx / (2 + p.r_v), m = idx % (2 + p.r_v);
+          p.partials[((bh0 + g) * p.S + r.s) * (2 + p.r_v) + m] = m == 0 ? -INFINITY : 0.f;
         }
       }
-      named_barrier(1, kEpiThreads);
-      for (int m = et; m < G * p.r_v; m += kEpiThreads) {
-        const int g = m / p.r_v, mm = m % p.r_v;
-        float acc = 0.f;
-        for (int q = 0; q < p.Q; ++q) acc += obuf[(q * G + g) * p.r_v + mm];
-        p.partials[((bh0 + g) * p.S + r.s) * (2 + p.r_v) + 2 + mm] = acc;
-      }
-      named_barrier(1, kEpiThreads);
     }
   }
 
@@ -669,25 +833,36 @@ int env_int(const char* name, int dflt) {
 
 struct TcPlan {
   bool ok = false;
-  int G = 1, nst = 0, nacc = 1, S = 0, tps = 0;
+  int G = 1, nst = 0, nst_v = 0, nacc = 1, S = 0, tps = 0;
   size_t ops_bytes = 0;   // workspace for the per-(b, h) operand images
 };
 
 // Shared-memory layout for (D, G, nst); returns total bytes (plus alignment slack).
-uint32_t tc_layout(TcParams& p, int D, int G, int nst) {
+uint32_t tc_layout(TcParams& p, int D, int G, int nst, int nst_v) {
   auto al = [](uint32_t x, uint32_t a) { return (x + a - 1) / a * a; };
   p.K_pad = (p.r_k + 15) / 16 * 16;
   p.box_k = p.K_pad % 64 == 0 ? 64 : (p.K_pad % 32 == 0 ? 32 : 16);
   p.nkb = p.K_pad / p.box_k;
   p.swz = p.box_k == 64 ? 2 : (p.box_k == 32 ? 4 : 6);
   p.box_bytes = kTile * p.box_k * 2;
-  p.cv_off = G * p.nkb * p.box_bytes;
-  p.st_bytes = al(p.cv_off + G * kTile * p.r_v * 2, 1024);
-  p.tx_bytes = p.cv_off + G * kTile * p.r_v * 2;
+  p.N_v = (p.r_v + 15) / 16 * 16;
+  p.cvb = p.N_v % 64 == 0 ? 64 : (p.N_v % 32 == 0 ? 32 : 16);
+  p.nvb = p.N_v / p.cvb;
+  p.swz_v = p.cvb == 64 ? 2 : (p.cvb == 32 ? 4 : 6);
+  p.vbox_bytes = kTile * p.cvb * 2;
+  p.nmb = (p.r_v + 127) / 128;
+  p.cv_off = 0;
+  p.tx_bytes = G * p.nkb * p.box_bytes;          // K latent stage
+  p.st_bytes = al(p.tx_bytes, 1024);
+  p.tx_v = G * p.nvb * p.vbox_bytes;             // V latent stage
+  p.stv_bytes = al(p.tx_v, 1024);
   p.nst = nst;
+  p.nst_v = nst_v;
   uint32_t o = 0;
   p.st_off = o;
   o += nst * p.st_bytes;
+  p.stv_off = o;
+  o += nst_v * p.stv_bytes;
   // two buffers of the query-absorbed B operand and of the bias tile (per item)
   p.b_off = o;
   p.b_head_bytes = D * p.K_pad * 2;
@@ -697,25 +872,19 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst) {
   p.bias_off = o;
   o = al(o + 2 * G * p.bias_head_bytes, 1024);
   p.ones_off = o;
-  o += 4096;
+  o += 256;
+  p.p_off = o;                       // softmax weights: 2 buffers x G x (8 rows x 128 tokens)
+  o += 2 * G * 8 * kTile * 2;
   p.sbuf_off = o;
-  o += (kEpiWG - 1) * G * kTile * 4;
-  p.p_off = o;
-  o += G * kTile * 4;
+  o += 2 * (kEpiWG - 1) * G * kTile * 4;
   p.red_off = o;
-  o += G * 4 * 4;
-  p.alpha_off = o;
-  o = al(o + G * 4, 16);
-  const int rv8 = p.r_v / 8;
-  int Q = kEpiThreads / (G * rv8);
-  if (Q < 1) Q = 1;
-  if (Q > 32) Q = 32;
-  p.Q = Q;
-  p.nv_items = G * rv8 * Q;
-  p.obuf_off = o;
-  o = al(o + Q * G * p.r_v * 4, 16);
+  o = al(o + G * 4 * 4, 16);
+  p.ctx_off = o;
+  o += kCtxCache * 4;
+  p.rope_off = o;            // float2 step[64], then uint2 phi[64]
+  o += 64 * 8 * 2;
   p.bar_off = o;
-  o += (2 * nst + 8) * 8;
+  o += (2 * nst + 2 * nst_v + 12) * 8;
   p.misc_off = o;
   o += 16;
   return o + 1024;
@@ -727,32 +896,45 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   if (c.mode != LLA_MODE_PER_HEAD || n_cap <= 0 || B <= 0) return pl;
   if (D != 32 && D != 64 && D != 96 && D != 128) return pl;
   const int forced_g = env_int("LLA_TC_G", 0), forced_nst = env_int("LLA_TC_NST", 0);
-  // Largest head group G whose ring fits at least 3 stages; else the largest with 2.
-  int best_g = 0, best_nst = 0;
+  const int N_v = (c.r_v + 15) / 16 * 16;
+  // Largest head group G whose TMEM columns (score accumulators plus V accumulators)
+  // fit in 512 and whose shared-memory ring holds at least 2 stages; two score
+  // buffers when they fit.
+  int best_g = 0, best_nst = 0, best_nst_v = 0, best_nacc = 1;
   for (int G : {4, 2, 1}) {
-    if (c.H % G || G * D > 512) continue;
+    if (c.H % G) continue;
     if (forced_g && G != forced_g) continue;
+    int nacc = 0;
+    const int vcols = G * N_v;
+    if (2 * G * D + vcols <= 512) nacc = 2;
+    else if (G * D + vcols <= 512) nacc = 1;
+    if (!nacc) continue;
     TcParams p{};
     p.r_k = c.r_k;
     p.r_v = c.r_v;
-    int nst = 0;
-    for (int s = 2; s <= 6; ++s)
-      if (tc_layout(p, D, G, s) <= kSmemLimit) nst = s;
+    // deepest V ring that fits (its slots are held longest), then the deepest K ring
+    int nst = 0, nst_v = 0;
+    for (int nv = 8; nv >= 2 && !nst; --nv)
+      for (int nk = 8; nk >= 2; --nk)
+        if (tc_layout(p, D, G, nk, nv) <= kSmemLimit) {
+          nst = nk;
+          nst_v = nv;
+          break;
+        }
     if (forced_nst && nst > forced_nst) nst = forced_nst;
-    if (nst >= 3) {
-      best_g = G;
-      best_nst = nst;
-      break;
-    }
-    if (nst >= 2 && best_g == 0) {
-      best_g = G;
-      best_nst = nst;
-    }
+    if (forced_nst && nst_v > forced_nst) nst_v = forced_nst;
+    if (nst < 2 || nst_v < 2) continue;
+    best_g = G;
+    best_nst = nst;
+    best_nst_v = nst_v;
+    best_nacc = nacc;
+    break;
   }
   if (!best_g) return pl;
   pl.G = best_g;
   pl.nst = best_nst;
-  pl.nacc = (2 * pl.G * D <= 512) ? 2 : 1;
+  pl.nst_v = best_nst_v;
+  pl.nacc = best_nacc;
   // Context splits: balance tiles over a 148-SM grid of persistent CTAs.
   const int n_tiles = (n_cap + kTile - 1) / kTile;
   const long long units = (long long)B * (c.H / pl.G);
@@ -848,7 +1030,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.r_k = a.r_k;
   p.r_v = a.r_v;
   // At least 120 KB so that two CTAs never share an SM (each may hold all of TMEM).
-  uint32_t smem = tc_layout(p, a.d, pl.G, pl.nst);
+  uint32_t smem = tc_layout(p, a.d, pl.G, pl.nst, pl.nst_v);
   if (smem < 120u * 1024u) smem = 120u * 1024u;
   p.B = a.B;
   p.n_cap = a.n_cap;
@@ -859,8 +1041,9 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.rope_max_pos = a.rope_max_pos;
   p.nacc = pl.nacc;
   p.acc_cols = pl.G * a.d;
+  p.v_col0 = p.nacc * p.acc_cols;
   int cols = 32;
-  while (cols < p.nacc * p.acc_cols) cols <<= 1;
+  while (cols < p.v_col0 + pl.G * p.N_v) cols <<= 1;
   p.tmem_cols = cols;
   p.rope = a.rope;
   for (int i = 0; i < a.d / 2; ++i) {
@@ -884,7 +1067,10 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!make_map(&mk, a.ck, a.H * a.r_k, a.n_cap, a.B, p.box_k, swz) ||
-      !make_map(&mv, a.cv, a.H * a.r_v, a.n_cap, a.B, a.r_v, CU_TENSOR_MAP_SWIZZLE_NONE))
+      !make_map(&mv, a.cv, a.H * a.r_v, a.n_cap, a.B, p.cvb,
+                p.cvb == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                : p.cvb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                              : CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorNotSupported;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
