@@ -31,6 +31,9 @@ import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = synth.WORKLOAD_ORDER[1]
 METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop step"
+# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu capture
+# summarised in profiles/decode_tc_perhead4x_B8_n4096.md; drop an entry when the kernel changes.
+NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 276.64e6}
 
 
 def parse():
@@ -286,7 +289,7 @@ def run_gpu(args):
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
         "roofline": {"bound": "hbm", "kernel": "lla_decode_attn (partial + combine)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get(w.name),
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "decode_call_us": round(dec_avg * 1e3, 2),
                      "algorithmic_bytes_per_call": decode_bytes(w, w.n)},
