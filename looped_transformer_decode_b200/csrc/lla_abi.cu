@@ -241,12 +241,15 @@ int lla_encode(const lla_cfg* cfg, const void* packed, int64_t n_tok, const uint
   PackedLayout L = packed_layout(*cfg);
   if (L.W > 49152)
     return fail(LLA_ERR_UNSUPPORTED, "encode input width %d above 49152", L.W);
-  cudaError_t ce = launch_encode(*cfg, L, static_cast<const char*>(packed), n_tok,
-                                 reinterpret_cast<const __nv_bfloat16*>(x_k),
-                                 reinterpret_cast<const __nv_bfloat16*>(x_v), slot, n_slots,
-                                 reinterpret_cast<__nv_bfloat16*>(c_k),
-                                 reinterpret_cast<__nv_bfloat16*>(c_v), status,
-                                 static_cast<cudaStream_t>(stream));
+  const char* pk = static_cast<const char*>(packed);
+  const auto* xk = reinterpret_cast<const __nv_bfloat16*>(x_k);
+  const auto* xv = reinterpret_cast<const __nv_bfloat16*>(x_v);
+  auto* ck = reinterpret_cast<__nv_bfloat16*>(c_k);
+  auto* cv = reinterpret_cast<__nv_bfloat16*>(c_v);
+  auto* st = static_cast<cudaStream_t>(stream);
+  cudaError_t ce = launch_encode_tc(*cfg, L, pk, n_tok, xk, xv, slot, n_slots, ck, cv, status, st);
+  if (ce == cudaErrorNotSupported)
+    ce = launch_encode(*cfg, L, pk, n_tok, xk, xv, slot, n_slots, ck, cv, status, st);
   if (ce != cudaSuccess) return cuda_fail(ce, "lla_encode launch");
   return ok();
 }

@@ -52,6 +52,11 @@ cudaError_t launch_encode(const lla_cfg& c, const PackedLayout& L, const char* p
                           int64_t n_tok, const __nv_bfloat16* xk, const __nv_bfloat16* xv,
                           const int64_t* slot, int64_t n_slots, __nv_bfloat16* ck,
                           __nv_bfloat16* cv, int32_t* status, cudaStream_t s);
+// Same contract on the tensor cores; cudaErrorNotSupported leaves the call to launch_encode.
+cudaError_t launch_encode_tc(const lla_cfg& c, const PackedLayout& L, const char* packed,
+                             int64_t n_tok, const __nv_bfloat16* xk, const __nv_bfloat16* xv,
+                             const int64_t* slot, int64_t n_slots, __nv_bfloat16* ck,
+                             __nv_bfloat16* cv, int32_t* status, cudaStream_t s);
 
 struct DecodeArgs {
   int T, H, d, r_k, r_v, mode;

@@ -6,9 +6,13 @@
 #pragma once
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 namespace lla {
+
+// cuTensorMapEncodeTiled from the driver, or null when it cannot be resolved.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 namespace sm100 {
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s

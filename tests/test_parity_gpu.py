@@ -41,16 +41,26 @@ ENCODE_CFGS = [
     O.Cfg(32, 2, 96, 64, 128),                    # deep loop, two heads
     O.Cfg(2, 4, 64, 32, 48, O.MODE_2D),           # LLA-2D small
     O.Cfg(4, 16, 128, 64, 128, O.MODE_2D),        # LLA-2D workload width
+    O.Cfg(3, 1, 96, 24, 40, O.MODE_2D),           # width 288: 32-wide K chunks, r not a multiple of 16
+    O.Cfg(8, 3, 32, 256, 8),                      # largest latent, smallest head
 ]
+ENCODE_PATHS = ["tensor_core", "cuda_core"]
 
 
+@pytest.mark.parametrize("path", ENCODE_PATHS)
+@pytest.mark.parametrize("n_tok", [37, 300])
 @pytest.mark.parametrize("cfg", ENCODE_CFGS, ids=lambda c: f"T{c.T}H{c.H}d{c.d}r{c.r_k}_{c.r_v}m{c.mode}")
-def test_encode_matches_oracle(cfg):
+def test_encode_matches_oracle(cfg, n_tok, path, monkeypatch):
+    """Both encode kernels against the oracle: one ragged 128-token tile, and three tiles."""
+    if path == "cuda_core":
+        monkeypatch.setenv("LLA_ENCODE_PATH", "cuda_core")
+    else:
+        monkeypatch.delenv("LLA_ENCODE_PATH", raising=False)
     case = decode_case(cfg, 1, 4, seed=50 + cfg.r_k, R=3)
     g = synth.rng(77)
     shared = cfg.mode == O.MODE_2D
     mk = synth.trajectory_model(g, cfg.T, cfg.H, cfg.d, 3, shared=shared)
-    n_tok, n_slots = 37, 50
+    n_slots = n_tok + 13
     xk = O.bf16_round(synth.sample_trajectories(g, mk, n_tok))
     xv = O.bf16_round(synth.sample_trajectories(g, mk, n_tok))
     slot = g.permutation(n_slots)[:n_tok]
