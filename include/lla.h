@@ -121,9 +121,10 @@ size_t lla_codec_packed_bytes(const lla_cfg* cfg);
  *   LLA-2D:    W_down_{k,v} [T*H*d][r],   W_up_{k,v} [T][H][d][r],  mu_{k,v} [T*H*d]
  *   (concatenation order: loop-major, then head for LLA-2D, then the d entries.)
  * The packed buffer (`packed`, device, >= lla_codec_packed_bytes(cfg)) holds W_up
- * and mu in fp32, W_down rounded to bf16 (round to nearest even), and the encode
- * bias mu W_down computed with that rounded W_down.  Inputs may be freed once the
- * stream has passed this call.
+ * and mu in fp32, W_down rounded to bf16 (round to nearest even; stored twice: row
+ * major, and cut into the tensor-core encode's operand tiles), and the encode bias
+ * mu W_down computed with that rounded W_down.  Inputs may be freed once the stream
+ * has passed this call.
  */
 int lla_codec_pack(const lla_cfg* cfg, const float* W_down_k, const float* W_down_v,
                    const float* W_up_k, const float* W_up_v, const float* mu_k,

@@ -93,6 +93,8 @@ PackedLayout packed_layout(const lla_cfg& c) {
   L.wdv = take((size_t)L.L * rv * L.W * 2);
   L.biask = take((size_t)L.L * rk * 4);
   L.biasv = take((size_t)L.L * rv * 4);
+  L.wimgk = take((size_t)L.L * pad16(c.r_k) * L.W * 2);
+  L.wimgv = take((size_t)L.L * pad16(c.r_v) * L.W * 2);
   L.total = o;
   return L;
 }

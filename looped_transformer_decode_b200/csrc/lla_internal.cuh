@@ -24,13 +24,26 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 //   mu_{k,v}   fp32 [T][H][d]         loop-t, head-h mean slice mu_t,h
 //   wd_{k,v}   bf16 [L][r][W]         W_down^T (rows = latent index), L = H (per head) or 1
 //   bias_{k,v} fp32 [L][r]            mu W_down with the bf16-rounded W_down
+//   wimg_{k,v} bf16 [L][W/kc][N][kc]  the same W_down^T cut into K chunks of kc entries,
+//                                     each chunk the swizzled K-major operand image of
+//                                     the tensor-core encode (N = r rounded up to 16,
+//                                     rows >= r zero), so that one bulk copy stages it
 struct PackedLayout {
-  size_t wupk, wupv, muk, muv, wdk, wdv, biask, biasv, total;
+  size_t wupk, wupv, muk, muv, wdk, wdv, biask, biasv, wimgk, wimgv, total;
   int L;     // latents per token and layer: H (per head) or 1 (LLA-2D)
   int W;     // encode input width: T*d (per head) or T*H*d (LLA-2D)
 };
 
 PackedLayout packed_layout(const lla_cfg& c);
+
+// K chunk (entries) of the tensor-core encode: 64 (128-byte swizzle) when a head's
+// d entries (per head) or the whole input row (LLA-2D) split into 64s, else 32
+// (64-byte swizzle).  Every supported d is a multiple of 32.
+inline int encode_kc(const lla_cfg& c) {
+  const int unit = c.mode == LLA_MODE_PER_HEAD ? c.d_head : c.T * c.H * c.d_head;
+  return unit % 64 == 0 ? 64 : 32;
+}
+inline int pad16(int r) { return (r + 15) / 16 * 16; }
 
 // Decode split plan shared by the workspace sizing and the launcher.
 struct SplitPlan {

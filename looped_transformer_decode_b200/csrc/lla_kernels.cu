@@ -138,6 +138,31 @@ __global__ void pack_bias_kernel(const float* __restrict__ mu, const __nv_bfloat
   if (lane == 0) bias[warp] = (float)acc;
 }
 
+// Tensor-core encode operand images.  Chunk c of latent l is the [N][kc] tile of
+// W_down^T (rows = latent index m, columns = input entries c*kc ...), rows >= r zero,
+// stored the way a swizzled K-major TMA box lands in shared memory: the 16-byte
+// unit u of row `row` (128-byte rows for kc = 64, 64-byte rows for kc = 32) sits at
+// unit u ^ (row-group bits 7.. of its byte offset), so one bulk copy stages it.
+__global__ void pack_wimg_kernel(const __nv_bfloat16* __restrict__ wd, __nv_bfloat16* __restrict__ img,
+                                 int L, int W, int r, int N, int kc) {
+  const int nch = W / kc;
+  const long long total = (long long)L * nch * N * kc;
+  const unsigned mask = kc == 64 ? 7u : 3u;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int col = (int)(e % kc);
+    const int row = (int)((e / kc) % N);
+    const long long tile = e / ((long long)kc * N);      // l * nch + c
+    const int c = (int)(tile % nch);
+    const int l = (int)(tile / nch);
+    const __nv_bfloat16 v = row < r ? wd[((long long)l * r + row) * W + (long long)c * kc + col]
+                                    : __float2bfloat16_rn(0.f);
+    const unsigned o = (unsigned)(row * kc + col) * 2u;
+    const unsigned so = o ^ (((o >> 7) & mask) << 4);
+    img[tile * N * kc + so / 2] = v;
+  }
+}
+
 // ---------------------------------------------------------------- encode
 
 // One CTA per (token, latent l, K or V).  c[m] = sum_k x[k] W^T[m][k] - bias[m].
@@ -458,6 +483,11 @@ cudaError_t launch_pack(const lla_cfg& c, const PackedLayout& L, const float* wd
   pack_wdown_kernel<<<512, 256, 0, s>>>(wdk, wdk_bf, L.L, L.W, c.r_k);
   pack_wdown_kernel<<<512, 256, 0, s>>>(wdv, wdv_bf, L.L, L.W, c.r_v);
   // mu in the input layout is already the concatenated mean per latent ([L][W]).
+  const int kc = encode_kc(c);
+  pack_wimg_kernel<<<512, 256, 0, s>>>(wdk_bf, reinterpret_cast<__nv_bfloat16*>(packed + L.wimgk),
+                                       L.L, L.W, c.r_k, pad16(c.r_k), kc);
+  pack_wimg_kernel<<<512, 256, 0, s>>>(wdv_bf, reinterpret_cast<__nv_bfloat16*>(packed + L.wimgv),
+                                       L.L, L.W, c.r_v, pad16(c.r_v), kc);
   const int wk = L.L * c.r_k, wv = L.L * c.r_v;
   pack_bias_kernel<<<(wk * 32 + 255) / 256, 256, 0, s>>>(
       muk, wdk_bf, reinterpret_cast<float*>(packed + L.biask), L.L, L.W, c.r_k);

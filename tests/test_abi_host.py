@@ -116,8 +116,9 @@ def test_encode_validation():
 def test_packed_and_rope_sizes():
     cfg = lla.Cfg(4, 16, 128, 96, 160)
     n = lla.lib.lla_codec_packed_bytes(ctypes.byref(cfg.c()))
-    # W_up and mu in fp32, W_down in bf16, bias in fp32 (each section 256-byte aligned)
-    want = (4 * 16 * 128 * (96 + 160) * 4 + 2 * 4 * 16 * 128 * 4 + 16 * (96 + 160) * 512 * 2
+    # W_up and mu in fp32, W_down in bf16 twice (row major and as encode operand tiles,
+    # rows padded to 16), bias in fp32; each section 256-byte aligned
+    want = (4 * 16 * 128 * (96 + 160) * 4 + 2 * 4 * 16 * 128 * 4 + 2 * 16 * (96 + 160) * 512 * 2
             + 16 * (96 + 160) * 4)
     assert want <= n < want + 8 * 256
     assert lla.lib.lla_rope_table_bytes(ctypes.byref(cfg.c()), 4097) == 4097 * 64 * 8

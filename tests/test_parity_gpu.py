@@ -44,18 +44,22 @@ ENCODE_CFGS = [
     O.Cfg(3, 1, 96, 24, 40, O.MODE_2D),           # width 288: 32-wide K chunks, r not a multiple of 16
     O.Cfg(8, 3, 32, 256, 8),                      # largest latent, smallest head
 ]
-ENCODE_PATHS = ["tensor_core", "cuda_core"]
+# tensor_core picks 128- or 256-token CTAs by size; tensor_core_m256 forces 256.
+ENCODE_PATHS = ["tensor_core", "tensor_core_m256", "cuda_core"]
 
 
 @pytest.mark.parametrize("path", ENCODE_PATHS)
 @pytest.mark.parametrize("n_tok", [37, 300])
 @pytest.mark.parametrize("cfg", ENCODE_CFGS, ids=lambda c: f"T{c.T}H{c.H}d{c.d}r{c.r_k}_{c.r_v}m{c.mode}")
 def test_encode_matches_oracle(cfg, n_tok, path, monkeypatch):
-    """Both encode kernels against the oracle: one ragged 128-token tile, and three tiles."""
+    """Both encode kernels against the oracle: one ragged 128-token tile, and three tiles
+    (two 256-token CTAs, the second one partly past the end, when forced)."""
+    monkeypatch.delenv("LLA_ENCODE_PATH", raising=False)
+    monkeypatch.delenv("LLA_ENC_MSUB", raising=False)
     if path == "cuda_core":
         monkeypatch.setenv("LLA_ENCODE_PATH", "cuda_core")
-    else:
-        monkeypatch.delenv("LLA_ENCODE_PATH", raising=False)
+    elif path == "tensor_core_m256":
+        monkeypatch.setenv("LLA_ENC_MSUB", "2")
     case = decode_case(cfg, 1, 4, seed=50 + cfg.r_k, R=3)
     g = synth.rng(77)
     shared = cfg.mode == O.MODE_2D
