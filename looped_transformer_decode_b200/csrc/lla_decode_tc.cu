@@ -1,4 +1,7 @@
-// Per-head LLA decode attention on the 5th-generation tensor cores (sm_100a).
+// LLA decode attention on the 5th-generation tensor cores (sm_100a), per head and
+// LLA-2D.  In LLA-2D every head reads the same latent row (close reading §二.6),
+// so the head offset into the latent is zero and a head group's tiles repeat the
+// same bytes, which L2 serves after the first read.
 //
 // Same arithmetic as the CUDA-core kernel (query folded into the K
 // up-projection, RoPE as a complex product with the fp64-built table, base-2
@@ -49,6 +52,7 @@ constexpr uint32_t kSmemLimit = 232448;  // per-block dynamic shared memory on s
 
 struct TcParams {
   int H, r_k, r_v, K_pad, box_k, nkb, swz;   // K latent tiles: K-major, swizzle code swz
+  int lat_hk, lat_hv;                        // latent columns between heads (0: LLA-2D, shared)
   int nst_v;                                 // V latent ring depth (nst: K latent ring)
   uint32_t stv_off, stv_bytes, tx_v;
   int N_v, cvb, nvb, swz_v;                  // V latent tiles: MN-major boxes of cvb dims
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int h = r.hg * G + g;
               for (int kb = 0; kb < p.nkb; ++kb)
                 tma_load_3d(st + (g * p.nkb + kb) * p.box_bytes, map, &fullb[stage],
-                            h * p.r_k + kb * p.box_k, y, r.b);
+                            h * p.lat_hk + kb * p.box_k, y, r.b);
             }
           } else {
             mbar_arrive_expect_tx(&fullb[stage], p.tx_v);
@@ -454,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int h = r.hg * G + g;
               for (int vb = 0; vb < p.nvb; ++vb)
                 tma_load_3d(st + (g * p.nvb + vb) * p.vbox_bytes, map, &fullb[stage],
-                            h * p.r_v + vb * p.cvb, y, r.b);
+                            h * p.lat_hv + vb * p.cvb, y, r.b);
             }
           }
         }
@@ -878,7 +882,7 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst, int nst_v) {
 TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   TcPlan pl;
   const int D = c.d_head;
-  if (c.mode != LLA_MODE_PER_HEAD || n_cap <= 0 || B <= 0) return pl;
+  if (n_cap <= 0 || B <= 0) return pl;
   if (D != 32 && D != 64 && D != 96 && D != 128) return pl;
   const int forced_g = env_int("LLA_TC_G", 0), forced_nst = env_int("LLA_TC_NST", 0);
   const int N_v = (c.r_v + 15) / 16 * 16;
@@ -1064,8 +1068,10 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   const CUtensorMapSwizzle swz = p.box_k == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (!make_map(&mk, a.ck, a.H * a.r_k, a.n_cap, a.B, p.box_k, swz) ||
-      !make_map(&mv, a.cv, a.H * a.r_v, a.n_cap, a.B, p.cvb,
+  p.lat_hk = (int)a.lat_head_k;
+  p.lat_hv = (int)a.lat_head_v;
+  if (!make_map(&mk, a.ck, (int)a.lat_tok_k, a.n_cap, a.B, p.box_k, swz) ||
+      !make_map(&mv, a.cv, (int)a.lat_tok_v, a.n_cap, a.B, p.cvb,
                 p.cvb == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                 : p.cvb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                               : CU_TENSOR_MAP_SWIZZLE_32B))
