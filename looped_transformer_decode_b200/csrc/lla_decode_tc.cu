@@ -63,6 +63,10 @@ struct TcParams {
       red_off, ctx_off, rope_off, bar_off, misc_off;
   int nst, nacc, acc_cols, v_col0, tmem_cols;
   uint32_t tx_bytes;
+  // LLA-2D kernel: B-operand buffers, P rows (N of the V MMA), 128-row blocks of r_v
+  int nbuf_b, n_p, m_v;
+  int poll;                                  // per-head hand-offs poll instead of suspending
+  uint32_t p_buf_bytes;
   const float2* rope;    // [rope_max_pos][d/2]
   const int32_t* ctx_len;
   const int32_t* positions;
@@ -112,6 +116,35 @@ __device__ __forceinline__ float warp_sum_f(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+// bar.red.or over the 128 threads of one warpgroup (named barrier `id`).
+__device__ __forceinline__ int wg_barrier_or(uint32_t id, int pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.red.or.pred po, %2, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred), "r"(id)
+      : "memory");
+  return static_cast<int>(out);
+}
+
+// bar.red.or over NT epilogue threads (named barrier 1): returns the OR of `pred`.
+template <int NT>
+__device__ __forceinline__ int epi_barrier_or_n(int pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "barrier.red.or.pred po, 1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(out)
+      : "r"(pred), "n"(NT)
+      : "memory");
+  return static_cast<int>(out);
 }
 
 // bar.red.or over the epilogue threads (named barrier 1): returns the OR of `pred`.
@@ -362,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], kEpiWarps);
       mbar_init(&bfull[a], 1);
       mbar_init(&bempty[a], 1);
-      mbar_init(&pfull[a], 1);
+      mbar_init(&pfull[a], 4);
       mbar_init(&pempty[a], 1);
     }
     *abort_flag = 0;
@@ -668,8 +701,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (wgi == 0) {
-          // ---- softmax weights against the item's reference maximum m_ref
+          // ---- softmax weights against the item's reference maximum m_ref, taken on
+          // the item's first tile; later tiles only check (one barrier) that no score
+          // exceeds it by more than 2^kRescaleLog2, and take a new maximum if one does
           float s[G];
+          int over = 0;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             float tot = part[g];
@@ -677,23 +713,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int w = 0; w < kEpiWG - 1; ++w)
               tot += sbuf[(((it & 1u) * (kEpiWG - 1) + w) * G + g) * kTile + row];
             s[g] = valid ? tot : -INFINITY;
-            const float mx = warp_max_f(s[g]);
-            if (lane == 0) red[g * 4 + sub] = mx;
+            over |= s[g] > m_ref[g] + kRescaleLog2;
           }
-          named_barrier(2, 128);
           bool rescale = false;
           float alpha[G];
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float mt = fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
-            alpha[g] = 1.f;
-            if (k == 0) {
-              m_ref[g] = mt;
-            } else if (mt > m_ref[g] + kRescaleLog2) {
-              alpha[g] = exp2f(m_ref[g] - mt);
-              m_ref[g] = mt;
-              rescale = true;
+          for (int g = 0; g < G; ++g) alpha[g] = 1.f;
+          if (k == 0 || wg_barrier_or(2, over)) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const float mx = warp_max_f(s[g]);
+              if (lane == 0) red[g * 4 + sub] = mx;
             }
+            named_barrier(2, 128);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const float mt =
+                  fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
+              if (k == 0) {
+                m_ref[g] = mt;
+              } else if (mt > m_ref[g] + kRescaleLog2) {
+                alpha[g] = exp2f(m_ref[g] - mt);
+                m_ref[g] = mt;
+                rescale = true;
+              }
+            }
+            named_barrier(2, 128);   // every warp has read red before it is reused
           }
           const uint32_t pb = it & 1u;
           // the weights buffer is free once the V MMA of tile it - 2 has finished
@@ -732,8 +777,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<__nv_bfloat16*>(pt + 16) = lo;
           }
           fence_proxy_async_smem();
-          named_barrier(2, 128);
-          if (row == 0) mbar_arrive(&pfull[pb]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pfull[pb]);   // one arrival per warp of the group
         }
         if (!ok) *abort_flag = 1;
         // off the critical path: RoPE factors of the next tile (its position was
@@ -799,6 +844,463 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
 }
 
+// LLA-2D: every head reads the same latent row (close reading §二.6), so a work
+// item (sequence b, group of HP heads, context split s) streams each 128-token
+// c_k and c_v tile once and uses it for all HP heads:
+//   * warp 1 issues the score MMAs head by head, U_h = C_k A~_h^T (+ bias), each
+//     into the next of nacc one-head TMEM buffers, so the epilogue drains head h
+//     while head h + 1 is multiplied;
+//   * warp 11 sums V transposed, D_v^T[r_v x 2 HP] += C_v^T P^T: the staged c_v
+//     tile is the MN-major A operand (M = 128 latent dims per block) and the
+//     softmax weights of all HP heads (rows 2g: hi, 2g + 1: lo) are the K-major
+//     B operand, so one set of K = 16 MMAs per tile serves the whole group.
+// The epilogue has four warpgroups, each owning a quarter of the RoPE pairs of
+// every token row (so a thread keeps 16 complex factors and the TMEM reads of a
+// head spread over 16 warps); warpgroup g also finalizes head g of the group:
+// its softmax, its weight rows, rescales and its partial.  Producers, bounded
+// waits and the abort path are those of decode_tc_kernel.
+constexpr int kEpiWG2 = 4;
+constexpr int kEpiThreads2 = 128 * kEpiWG2;
+constexpr int kEpiWarps2 = kEpiThreads2 / 32;
+constexpr int kThreads2 = 64 + kEpiThreads2 + 64;
+constexpr int kVProdWarp2 = 2 + kEpiWarps2, kVMmaWarp2 = 3 + kEpiWarps2;
+
+template <int D, int HP>
+__global__ void __launch_bounds__(kThreads2, 1)
+    decode_tc2d_kernel(const __grid_constant__ CUtensorMap map_k,
+                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
+  constexpr int HALF = D / 2;
+  constexpr int WG_PAIRS = HALF / kEpiWG2;
+  static_assert(HP <= kEpiWG2, "one finalizing warpgroup per head");
+  constexpr int WG_COLS = 2 * WG_PAIRS;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(sm + p.bar_off);   // [nst]
+  uint64_t* empty_k = full_k + p.nst;                                // [nst]
+  uint64_t* full_v = empty_k + p.nst;                                // [nst_v]
+  uint64_t* empty_v = full_v + p.nst_v;                              // [nst_v]
+  uint64_t* tfull = empty_v + p.nst_v;   // [nacc] one head's scores in TMEM
+  uint64_t* tempty = tfull + 4;          // [nacc] scores read
+  uint64_t* bfull = tempty + 4;          // [nbuf_b] query-absorbed operands loaded
+  uint64_t* bempty = bfull + 2;          // [nbuf_b] operand buffer free
+  uint64_t* pfull = bempty + 2;          // [2] softmax weights written
+  uint64_t* pempty = pfull + 2;          // [2] V MMA done with the weights buffer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ops_head_bytes = p.b_head_bytes;
+  const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.nst; ++s) {
+      mbar_init(&full_k[s], 1);
+      mbar_init(&empty_k[s], 1);
+    }
+    for (int s = 0; s < p.nst_v; ++s) {
+      mbar_init(&full_v[s], 1);
+      mbar_init(&empty_v[s], 1);
+    }
+    for (int a = 0; a < p.nacc; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiWarps2);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bfull[a], 1);
+      mbar_init(&bempty[a], 1);
+      mbar_init(&pfull[a], 4 * HP);
+      mbar_init(&pempty[a], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp >= 2 && warp < 2 + kEpiWarps2) {
+    const int et = threadIdx.x - 64;
+    if (ctx_s) {
+      int* cs = reinterpret_cast<int*>(sm + p.ctx_off);
+      for (int b = et; b < p.B; b += kEpiThreads2) {
+        int n = p.ctx_len[b];
+        if (n < 0 || n > p.n_cap) {
+          if (blockIdx.x == 0) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
+          n = n < 0 ? 0 : p.n_cap;
+        }
+        cs[b] = n;
+      }
+    }
+    if (et < 64) {
+      reinterpret_cast<float2*>(sm + p.rope_off)[et] = p.step[et];
+      reinterpret_cast<uint2*>(sm + p.rope_off + 512)[et] = make_uint2(p.phi_lo[et], p.phi_hi[et]);
+    }
+    if (et < 8 * 16) {
+      const int m = et / 16, k = et % 16;
+      *reinterpret_cast<__nv_bfloat16*>(sm + p.ones_off + (k >> 3) * 128 + m * 16 + (k & 7) * 2) =
+          __float2bfloat16_rn(k < 2 ? 1.f : 0.f);
+    }
+    // both weight buffers start zero: rows >= 2 HP are never written
+    for (int idx = et; idx < 2 * (int)p.p_buf_bytes / 4; idx += kEpiThreads2)
+      reinterpret_cast<uint32_t*>(sm + p.p_off)[idx] = 0u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 || warp == kVProdWarp2) {
+    // ------------------------------------------------------------ TMA producers
+    if (lane == 0) {
+      const bool kside = warp == 0;
+      const CUtensorMap* map = kside ? &map_k : &map_v;
+      tma_prefetch_desc(map);
+      const int nst = kside ? p.nst : p.nst_v;
+      uint64_t* fullb = kside ? full_k : full_v;
+      uint64_t* emptyb = kside ? empty_k : empty_v;
+      uint32_t it = 0, jn = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        if (r.ntiles == 0) continue;
+        if (kside) {
+          const uint32_t buf = jn % p.nbuf_b, bph = (jn / p.nbuf_b) & 1u;
+          if (!mbar_wait(&bempty[buf], bph ^ 1u, abort_flag)) break;
+          const size_t head0 = (size_t)r.b * p.H + (size_t)r.hg * HP;
+          mbar_arrive_expect_tx(&bfull[buf], HP * (ops_head_bytes + p.bias_head_bytes));
+          bulk_load(sm + p.b_off + buf * HP * ops_head_bytes, p.ops_b + head0 * ops_head_bytes,
+                    HP * ops_head_bytes, &bfull[buf]);
+          bulk_load(sm + p.bias_off + buf * HP * p.bias_head_bytes,
+                    p.ops_bias + head0 * p.bias_head_bytes, HP * p.bias_head_bytes, &bfull[buf]);
+          ++jn;
+        }
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t stage = it % nst, ph = (it / nst) & 1u;
+          if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int y = r.tok0 + k * kTile;
+          if (kside) {
+            mbar_arrive_expect_tx(&fullb[stage], p.tx_bytes);
+            unsigned char* st = sm + p.st_off + stage * p.st_bytes;
+            for (int kb = 0; kb < p.nkb; ++kb)
+              tma_load_3d(st + kb * p.box_bytes, map, &fullb[stage], kb * p.box_k, y, r.b);
+          } else {
+            mbar_arrive_expect_tx(&fullb[stage], p.tx_v);
+            unsigned char* st = sm + p.stv_off + stage * p.stv_bytes;
+            for (int vb = 0; vb < p.nvb; ++vb)
+              tma_load_3d(st + vb * p.vbox_bytes, map, &fullb[stage], vb * p.cvb, y, r.b);
+          }
+        }
+      }
+      if (*abort_flag) {
+        const uint32_t n_out = it < (uint32_t)nst ? it : (uint32_t)nst;
+        for (uint32_t j = 0; j < n_out; ++j) {
+          const uint32_t i = it - 1 - j;
+          const uint32_t stage = i % nst, ph = (i / nst) & 1u;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&fullb[stage], ph) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+        for (uint32_t j = 0; kside && j < (uint32_t)p.nbuf_b && j < jn; ++j) {
+          const uint32_t i = jn - 1 - j;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&bfull[i % p.nbuf_b], (i / p.nbuf_b) & 1u) &&
+                 global_timer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ score MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D);
+      const uint32_t sbo_a = 16u * p.box_k;
+      const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 0, 0);   // rows alias
+      uint32_t it = 0, jn = 0, u = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        if (r.ntiles == 0) continue;
+        const uint32_t buf = jn % p.nbuf_b, bph = (jn / p.nbuf_b) & 1u;
+        if (!mbar_wait(&bfull[buf], bph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ++jn;
+        const uint32_t b_base = smem_addr(sm + p.b_off + buf * HP * ops_head_bytes);
+        const uint32_t bias_base = smem_addr(sm + p.bias_off + buf * HP * p.bias_head_bytes);
+        for (int k = 0; ok && k < r.ntiles; ++k, ++it) {
+          const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
+          if (!mbar_wait(&full_k[stage], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st_addr = smem_addr(sm + p.st_off + stage * p.st_bytes);
+#pragma unroll 1
+          for (int g = 0; g < HP; ++g, ++u) {
+            const uint32_t acc = u % p.nacc, aph = (u / p.nacc) & 1u;
+            if (!(p.poll ? mbar_wait_poll(&tempty[acc], aph ^ 1u, abort_flag)
+                         : mbar_wait(&tempty[acc], aph ^ 1u, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * D;
+            const uint32_t b_addr = b_base + g * ops_head_bytes;
+            for (int kk = 0; kk < p.K_pad / 16; ++kk) {
+              const int kb = (kk * 16) / p.box_k, kin = (kk * 16) % p.box_k;
+              const uint64_t adesc =
+                  smem_desc(st_addr + kb * p.box_bytes + kin * 2, 16, sbo_a, p.swz);
+              const uint64_t bdesc = smem_desc(b_addr + kk * 256, 128, p.b_sbo, 0);
+              mma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            }
+            const uint64_t bias_desc = smem_desc(bias_base + g * p.bias_head_bytes, 128, 256, 0);
+            mma_bf16(d_tmem, odesc, bias_desc, idesc, 1u);
+            mma_commit(&tfull[acc]);
+          }
+          if (!ok) break;
+          mma_commit(&empty_k[stage]);
+          if (k == r.ntiles - 1) mma_commit(&bempty[buf]);   // last use of this B buffer
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kVMmaWarp2) {
+    // ------------------------------------------------------------ V MMA issuer
+    // D_v^T[block mb] (+)= C_v^T (128 latent dims x 128 tokens, MN-major A) x P^T
+    // (128 tokens x n_p weight rows, K-major B): one K=16 MMA per 16 tokens.
+    if (lane == 0) {
+      const uint32_t idesc_v = idesc_bf16_f32(128, p.n_p) | (1u << 15);   // A (c_v) MN-major
+      const uint32_t sbo_v = 16u * p.cvb;          // 8 token rows of one MN box
+      const uint32_t boxes_per_block = 128u / p.cvb;
+      const uint32_t p_base = smem_addr(sm + p.p_off);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t pb = it & 1u;
+          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag) ||
+              !mbar_wait(&full_v[vs], vph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t cv_addr = smem_addr(sm + p.stv_off + vs * p.stv_bytes);
+          const uint32_t b_addr = p_base + pb * p.p_buf_bytes;
+          for (int mb = 0; mb < p.m_v; ++mb) {
+            const uint32_t d_tmem = tmem_base + p.v_col0 + mb * p.n_p;
+            const uint32_t a_addr = cv_addr + mb * boxes_per_block * p.vbox_bytes;
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t adesc =
+                  smem_desc(a_addr + kk * 2 * sbo_v, p.vbox_bytes, sbo_v, p.swz_v);
+              const uint64_t bdesc = smem_desc(b_addr + kk * 256, 128, 2048, 0);
+              mma_bf16(d_tmem, adesc, bdesc, idesc_v, (k == 0 && kk == 0) ? 0u : 1u);
+            }
+          }
+          mma_commit(&pempty[pb]);
+          mma_commit(&empty_v[vs]);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;
+    const int wgi = (warp - 2) >> 2;          // quarter of the RoPE pairs; head it finalizes
+    const int sub = warp & 3;                 // TMEM sub-partition of this warp
+    const int row = sub * 32 + lane;          // token row of the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+    const bool fin = wgi < HP;                // this warpgroup finalizes head wgi
+    float* sbuf = reinterpret_cast<float*>(sm + p.sbuf_off);   // [2][HP][kEpiWG2][128]
+    float* red = reinterpret_cast<float*>(sm + p.red_off);     // [HP][4]
+
+    TileCursor pc;
+    cursor_first(p, ctx_s, pc);
+    float2 ef[WG_PAIRS];
+    int pos_cur = kNoPos, run = 0;
+    const float2* step_s = reinterpret_cast<const float2*>(sm + p.rope_off) + wgi * WG_PAIRS;
+    const uint2* phi_s = reinterpret_cast<const uint2*>(sm + p.rope_off + 512) + wgi * WG_PAIRS;
+    auto advance_rope = [&](int praw) {
+      if (praw == kNoPos) return;
+      const int pn = checked_pos(p, praw);
+      if (pos_cur != kNoPos && pn == pos_cur + kTile && run < kReseedTiles) {
+#pragma unroll
+        for (int q = 0; q < WG_PAIRS; ++q) {
+          const float2 st = step_s[q];
+          const float2 e = ef[q];
+          ef[q] = make_float2(fmaf(e.x, st.x, -e.y * st.y), fmaf(e.x, st.y, e.y * st.x));
+        }
+        ++run;
+      } else {
+#pragma unroll
+        for (int q = 0; q < WG_PAIRS; ++q) {
+          const uint2 ph = phi_s[q];
+          ef[q] = rope_factor(static_cast<uint32_t>(pn), ph.x, ph.y);
+        }
+        run = 0;
+      }
+      pos_cur = pn;
+    };
+#pragma unroll
+    for (int q = 0; q < WG_PAIRS; ++q) ef[q] = make_float2(1.f, 0.f);
+    advance_rope(cursor_pos(p, pc, row));
+    cursor_next(p, ctx_s, pc);
+    int pos_next = cursor_pos(p, pc, row);
+    cursor_next(p, ctx_s, pc);
+
+    uint32_t it = 0, u = 0;
+    bool aborted = false;
+    for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
+      const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
+      float m_ref = -INFINITY, l_part = 0.f;  // head wgi of the group (finalizing warpgroups)
+      for (int k = 0; k < r.ntiles; ++k, ++it) {
+        const int t0 = r.tok0 + k * kTile;
+        const int cnt = min(kTile, r.tok_end - t0);
+        const bool valid = row < cnt;
+        const uint32_t par = it & 1u;
+        bool ok = true;
+#pragma unroll 1
+        for (int g = 0; g < HP; ++g, ++u) {
+          const uint32_t acc = u % p.nacc, aph = (u / p.nacc) & 1u;
+          ok = ok && (p.poll ? mbar_wait_poll(&tfull[acc], aph, abort_flag)
+                             : mbar_wait(&tfull[acc], aph, abort_flag));
+          tc_fence_after();
+          float uu[WG_COLS];
+          const uint32_t col = tmem_base + lane_addr + acc * D + wgi * WG_COLS;
+#pragma unroll
+          for (int c = 0; c < WG_COLS / 16; ++c) tmem_ld16(col + c * 16, uu + c * 16);
+          if constexpr (WG_COLS % 16 != 0)
+            tmem_ld8(col + (WG_COLS / 16) * 16, uu + (WG_COLS / 16) * 16);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+          float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < WG_PAIRS; q += 2) {
+            a0 = ffma2(make_float2(uu[2 * q], uu[2 * q + 1]), ef[q], a0);
+            if (q + 1 < WG_PAIRS) a1 = ffma2(make_float2(uu[2 * q + 2], uu[2 * q + 3]), ef[q + 1], a1);
+          }
+          sbuf[((par * HP + g) * kEpiWG2 + wgi) * kTile + row] = (a0.x + a0.y) + (a1.x + a1.y);
+        }
+        if (epi_barrier_or_n<kEpiThreads2>(!ok)) {
+          aborted = true;
+          break;
+        }
+        if (fin) {
+          // ---- softmax weights of head wgi against the item's reference maximum
+          const int g = wgi;
+          float tot = 0.f;
+#pragma unroll
+          for (int w = 0; w < kEpiWG2; ++w) tot += sbuf[((par * HP + g) * kEpiWG2 + w) * kTile + row];
+          const float sc = valid ? tot : -INFINITY;
+          float alpha = 1.f;
+          bool rescale = false;
+          // reference maximum on the item's first tile; later tiles take a new one only
+          // when a score exceeds it by more than 2^kRescaleLog2 (one barrier to check)
+          if (k == 0 || wg_barrier_or(2 + wgi, sc > m_ref + kRescaleLog2)) {
+            const float mx = warp_max_f(sc);
+            if (lane == 0) red[g * 4 + sub] = mx;
+            named_barrier(2 + wgi, 128);
+            const float mt =
+                fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
+            if (k == 0) {
+              m_ref = mt;
+            } else if (mt > m_ref + kRescaleLog2) {
+              alpha = exp2f(m_ref - mt);
+              m_ref = mt;
+              rescale = true;
+            }
+            named_barrier(2 + wgi, 128);
+          }
+          const uint32_t pb = it & 1u;
+          // the weights buffer is free once the V MMA of tile it - 2 has finished
+          ok = mbar_wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u, abort_flag);
+          if (rescale) {
+            // rare: rescale head g's V accumulator columns 2g, 2g + 1 in every lane once
+            // the V MMA of the previous tile has finished; each warp owns its 32 lanes
+            ok = ok && mbar_wait(&pempty[(it - 1) & 1u], ((it - 1) >> 1) & 1u, abort_flag);
+            tc_fence_after();
+            for (int mb = 0; mb < p.m_v; ++mb) {
+              const uint32_t ta = tmem_base + lane_addr + p.v_col0 + mb * p.n_p + 2 * g;
+              float v[2];
+              tmem_ld2(ta, v);
+              tmem_wait_ld();
+              tmem_st2(ta, v[0] * alpha, v[1] * alpha);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+          }
+          const float pj = valid ? exp2f(sc - m_ref) : 0.f;
+          l_part = l_part * alpha + pj;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(pj);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(pj - __bfloat162float(hi));
+          // weight rows 2g (hi) and 2g + 1 (lo): row group (2g) / 8, rows (2g) % 8 and + 1
+          unsigned char* pg = sm + p.p_off + pb * p.p_buf_bytes + ((2 * g) >> 3) * 2048 +
+                              (row >> 3) * 128 + ((2 * g) & 7) * 16 + (row & 7) * 2;
+          *reinterpret_cast<__nv_bfloat16*>(pg) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(pg + 16) = lo;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pfull[pb]);   // one arrival per warp of the group
+        }
+        if (!ok) *abort_flag = 1;
+        advance_rope(pos_next);
+        pos_next = cursor_pos(p, pc, row);
+        cursor_next(p, ctx_s, pc);
+      }
+      if (aborted) break;
+      // ---------------------------------------------------------- item partial
+      if (fin && r.ntiles > 0) {
+        const int g = wgi;
+        const size_t bh = (size_t)r.b * p.H + r.hg * HP + g;
+        float* part_out = p.partials + (bh * p.S + r.s) * (2 + p.r_v);
+        const float l = warp_sum_f(l_part);
+        if (lane == 0) red[g * 4 + sub] = l;
+        const uint32_t last = it - 1;
+        const bool okv =
+            __all_sync(0xffffffffu, mbar_wait(&pempty[last & 1u], (last >> 1) & 1u, abort_flag));
+        tc_fence_after();
+        named_barrier(2 + wgi, 128);
+        if (okv) {
+          if (row == 0) {
+            part_out[0] = m_ref;
+            part_out[1] = red[g * 4] + red[g * 4 + 1] + red[g * 4 + 2] + red[g * 4 + 3];
+          }
+          for (int mb = 0; mb < p.m_v; ++mb) {
+            float v[2];
+            tmem_ld2(tmem_base + lane_addr + p.v_col0 + mb * p.n_p + 2 * g, v);
+            tmem_wait_ld();
+            const int m = mb * 128 + row;            // latent dim held by this lane
+            if (m < p.r_v) part_out[2 + m] = v[0] + v[1];
+          }
+        }
+        tc_fence_before();
+        named_barrier(2 + wgi, 128);
+      } else if (fin) {
+        const size_t bh = (size_t)r.b * p.H + r.hg * HP + wgi;
+        for (int m = row; m < 2 + p.r_v; m += 128)
+          p.partials[(bh * p.S + r.s) * (2 + p.r_v) + m] = m == 0 ? -INFINITY : 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+}
+
 // ------------------------------------------------------------------ host side
 
 bool make_map(CUtensorMap* map, const void* base, int inner, int n_cap, int B, int box_inner,
@@ -822,7 +1324,8 @@ int env_int(const char* name, int dflt) {
 
 struct TcPlan {
   bool ok = false;
-  int G = 1, nst = 0, nst_v = 0, nacc = 1, S = 0, tps = 0;
+  bool shared = false;    // LLA-2D kernel (G heads per item share each latent tile)
+  int G = 1, nst = 0, nst_v = 0, nacc = 1, nbuf_b = 2, S = 0, tps = 0;
   size_t ops_bytes = 0;   // workspace for the per-(b, h) operand images
 };
 
@@ -879,6 +1382,62 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst, int nst_v) {
   return o + 1024;
 }
 
+// Shared-memory layout of the LLA-2D kernel for (D, HP heads, rings, B buffers).
+uint32_t tc2d_layout(TcParams& p, int D, int HP, int nst, int nst_v, int nbuf_b) {
+  auto al = [](uint32_t x, uint32_t a) { return (x + a - 1) / a * a; };
+  p.K_pad = (p.r_k + 15) / 16 * 16;
+  p.box_k = p.K_pad % 64 == 0 ? 64 : (p.K_pad % 32 == 0 ? 32 : 16);
+  p.nkb = p.K_pad / p.box_k;
+  p.swz = p.box_k == 64 ? 2 : (p.box_k == 32 ? 4 : 6);
+  p.box_bytes = kTile * p.box_k * 2;
+  p.N_v = (p.r_v + 15) / 16 * 16;
+  p.cvb = p.N_v % 64 == 0 ? 64 : (p.N_v % 32 == 0 ? 32 : 16);
+  p.nvb = p.N_v / p.cvb;
+  p.swz_v = p.cvb == 64 ? 2 : (p.cvb == 32 ? 4 : 6);
+  p.vbox_bytes = kTile * p.cvb * 2;
+  p.m_v = (p.N_v + 127) / 128;
+  p.n_p = (2 * HP + 15) / 16 * 16;
+  p.p_buf_bytes = (uint32_t)p.n_p * kTile * 2;
+  p.tx_bytes = p.nkb * p.box_bytes;
+  p.st_bytes = al(p.tx_bytes, 1024);
+  p.tx_v = p.nvb * p.vbox_bytes;
+  // V stages span whole 128-row blocks of the MN-major A operand; the rows past
+  // r_v only feed TMEM lanes that are never read.
+  p.stv_bytes = al(p.m_v * (128 / p.cvb) * p.vbox_bytes, 1024);
+  p.nst = nst;
+  p.nst_v = nst_v;
+  p.nbuf_b = nbuf_b;
+  uint32_t o = 0;
+  p.st_off = o;
+  o += nst * p.st_bytes;
+  p.stv_off = o;
+  o += nst_v * p.stv_bytes;
+  p.b_off = o;
+  p.b_head_bytes = D * p.K_pad * 2;
+  p.b_sbo = (p.K_pad / 8) * 128;
+  o = al(o + nbuf_b * HP * p.b_head_bytes, 1024);
+  p.bias_head_bytes = D * 16 * 2;
+  p.bias_off = o;
+  o = al(o + nbuf_b * HP * p.bias_head_bytes, 1024);
+  p.ones_off = o;
+  o += 256;
+  p.p_off = o;
+  o += 2 * p.p_buf_bytes;
+  p.sbuf_off = o;
+  o += 2 * kEpiWG2 * HP * kTile * 4;
+  p.red_off = o;
+  o = al(o + HP * 4 * 4, 16);
+  p.ctx_off = o;
+  o += kCtxCache * 4;
+  p.rope_off = o;
+  o += 64 * 8 * 2;
+  p.bar_off = o;
+  o += (2 * nst + 2 * nst_v + 16) * 8;
+  p.misc_off = o;
+  o += 16;
+  return o + 1024;
+}
+
 TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   TcPlan pl;
   const int D = c.d_head;
@@ -890,7 +1449,42 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   // fit in 512 and whose shared-memory ring holds at least 2 stages; two score
   // buffers when they fit.
   int best_g = 0, best_nst = 0, best_nst_v = 0, best_nacc = 1;
+  if (c.mode == LLA_MODE_2D) {
+    // HP heads per item share each latent tile: the largest HP whose operands fit,
+    // double-buffered when possible; three one-head score buffers when TMEM allows.
+    for (int HP : {4, 2, 1}) {
+      if (c.H % HP || best_g) continue;
+      if (forced_g && HP != forced_g) continue;
+      const int m_v = (N_v + 127) / 128, n_p = (2 * HP + 15) / 16 * 16;
+      const int nacc = 3 * D + m_v * n_p <= 512 ? 3 : (2 * D + m_v * n_p <= 512 ? 2 : 0);
+      if (!nacc) continue;
+      for (int nbuf : {2, 1}) {
+        TcParams p{};
+        p.r_k = c.r_k;
+        p.r_v = c.r_v;
+        int nst = 0, nst_v = 0;
+        for (int nv = 6; nv >= 2 && !nst; --nv)
+          for (int nk = 6; nk >= 2; --nk)
+            if (tc2d_layout(p, D, HP, nk, nv, nbuf) <= kSmemLimit) {
+              nst = nk;
+              nst_v = nv;
+              break;
+            }
+        if (forced_nst && nst > forced_nst) nst = forced_nst;
+        if (forced_nst && nst_v > forced_nst) nst_v = forced_nst;
+        if (nst < 2 || nst_v < 2) continue;
+        best_g = HP;
+        best_nst = nst;
+        best_nst_v = nst_v;
+        best_nacc = nacc;
+        pl.nbuf_b = nbuf;
+        pl.shared = true;
+        break;
+      }
+    }
+  }
   for (int G : {4, 2, 1}) {
+    if (pl.shared) break;
     if (c.H % G) continue;
     if (forced_g && G != forced_g) continue;
     int nacc = 0;
@@ -955,23 +1549,26 @@ bool tc_enabled() {
   return !(v && std::strcmp(v, "cuda_core") == 0);
 }
 
-template <int D, int G>
+template <int D, int G, bool SHARED>
 cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
                         uint32_t smem, int grid, cudaStream_t s) {
-  auto kern = decode_tc_kernel<D, G>;
+  auto kern = SHARED ? decode_tc2d_kernel<D, G> : decode_tc_kernel<D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, s>>>(mk, mv, p);
+  kern<<<grid, SHARED ? kThreads2 : kThreads, smem, s>>>(mk, mv, p);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_tc_d(int G, const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
-                        uint32_t smem, int grid, cudaStream_t s) {
-  switch (G) {
-    case 1: return launch_tc_t<D, 1>(mk, mv, p, smem, grid, s);
-    case 2: return launch_tc_t<D, 2>(mk, mv, p, smem, grid, s);
-    case 4: return launch_tc_t<D, 4>(mk, mv, p, smem, grid, s);
+cudaError_t launch_tc_d(int G, bool shared, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
+  switch (G * 2 + (shared ? 1 : 0)) {
+    case 2: return launch_tc_t<D, 1, false>(mk, mv, p, smem, grid, s);
+    case 4: return launch_tc_t<D, 2, false>(mk, mv, p, smem, grid, s);
+    case 8: return launch_tc_t<D, 4, false>(mk, mv, p, smem, grid, s);
+    case 3: return launch_tc_t<D, 1, true>(mk, mv, p, smem, grid, s);
+    case 5: return launch_tc_t<D, 2, true>(mk, mv, p, smem, grid, s);
+    case 9: return launch_tc_t<D, 4, true>(mk, mv, p, smem, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1032,7 +1629,8 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.r_k = a.r_k;
   p.r_v = a.r_v;
   // At least 120 KB so that two CTAs never share an SM (each may hold all of TMEM).
-  uint32_t smem = tc_layout(p, a.d, pl.G, pl.nst, pl.nst_v);
+  uint32_t smem = pl.shared ? tc2d_layout(p, a.d, pl.G, pl.nst, pl.nst_v, pl.nbuf_b)
+                            : tc_layout(p, a.d, pl.G, pl.nst, pl.nst_v);
   if (smem < 120u * 1024u) smem = 120u * 1024u;
   p.B = a.B;
   p.n_cap = a.n_cap;
@@ -1042,10 +1640,11 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.n_items = a.B * p.HG * pl.S;
   p.rope_max_pos = a.rope_max_pos;
   p.nacc = pl.nacc;
-  p.acc_cols = pl.G * a.d;
+  p.acc_cols = pl.shared ? a.d : pl.G * a.d;
   p.v_col0 = p.nacc * p.acc_cols;
+  const int v_cols = pl.shared ? p.m_v * p.n_p : pl.G * p.N_v;
   int cols = 32;
-  while (cols < p.v_col0 + pl.G * p.N_v) cols <<= 1;
+  while (cols < p.v_col0 + v_cols) cols <<= 1;
   p.tmem_cols = cols;
   p.rope = a.rope;
   for (int i = 0; i < a.d / 2; ++i) {
@@ -1068,6 +1667,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   const CUtensorMapSwizzle swz = p.box_k == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
+  p.poll = env_int("LLA_TC_POLL", 1);
   p.lat_hk = (int)a.lat_head_k;
   p.lat_hv = (int)a.lat_head_v;
   if (!make_map(&mk, a.ck, (int)a.lat_tok_k, a.n_cap, a.B, p.box_k, swz) ||
@@ -1083,10 +1683,10 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   if (pe != cudaSuccess) return pe;
   const int grid = p.n_items < sms ? p.n_items : sms;
   switch (a.d) {
-    case 32: return launch_tc_d<32>(pl.G, mk, mv, p, smem, grid, s);
-    case 64: return launch_tc_d<64>(pl.G, mk, mv, p, smem, grid, s);
-    case 96: return launch_tc_d<96>(pl.G, mk, mv, p, smem, grid, s);
-    case 128: return launch_tc_d<128>(pl.G, mk, mv, p, smem, grid, s);
+    case 32: return launch_tc_d<32>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
+    case 64: return launch_tc_d<64>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
+    case 96: return launch_tc_d<96>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
+    case 128: return launch_tc_d<128>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
     default: return cudaErrorNotSupported;
   }
 }

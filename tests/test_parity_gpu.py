@@ -119,6 +119,11 @@ SMALL = [
     (O.Cfg(4, 2, 64, 16, 32), 2, 260, None, {"positions": "random"}),            # arbitrary positions
     (O.Cfg(2, 4, 64, 32, 48, O.MODE_2D), 2, 200, [200, 77], {}),                 # LLA-2D
     (O.Cfg(4, 4, 128, 64, 128, O.MODE_2D), 1, 300, None, {"q_scale": 10.0}),
+    # LLA-2D head groups of 2 (H = 6) and 1 (H = 3), r_v above 128 (two row blocks of
+    # the transposed V sum), small d, ragged and empty contexts, arbitrary positions
+    (O.Cfg(4, 6, 96, 48, 160, O.MODE_2D), 2, 260, [260, 131], {}),
+    (O.Cfg(2, 3, 32, 16, 24, O.MODE_2D), 3, 140, [140, 1, 0], {}),
+    (O.Cfg(4, 8, 64, 32, 64, O.MODE_2D), 2, 390, None, {"positions": "random", "q_scale": 20.0}),
 ]
 
 
