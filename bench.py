@@ -15,6 +15,7 @@ sample of the same workload (the reference arm of this benchmark).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import subprocess
@@ -33,7 +34,10 @@ DEFAULT_WORKLOAD = synth.WORKLOAD_ORDER[1]
 METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop step"
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu capture
 # summarised in profiles/decode_tc_perhead4x_B8_n4096.md; drop an entry when the kernel changes.
-NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 276.64e6}
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of the
+# current kernels (profiles/); a workload without a capture of the current code reports null.
+NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 277.10e6,
+               "lla2d_T4_H16_d128_r64_128_B512_n4096": 989.49e6}
 
 
 def parse():
@@ -46,6 +50,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--encode-tokens", type=int, default=0,
+                   help="override the workload's tokens encoded per step (profiling aid)")
     return p.parse_args()
 
 
@@ -81,17 +87,40 @@ def peaks():
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
+    """nvidia-smi clocks and throttle reasons every 20 ms, with host timestamps.
+
+    Started before the last warm-up steps (nvidia-smi needs a few hundred ms to
+    produce its first line); only the samples taken inside the timed region are
+    kept, or, when that region is shorter than the sampling period, the samples
+    nearest to it (the GPU is busy with the same steps on both sides).
+    """
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
     def __init__(self, gpu_index: int):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        self.t0 = self.t1 = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-i", str(gpu_index), "-lms", "20"], stdout=self.f,
-                                      stderr=subprocess.DEVNULL)
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-i", str(gpu_index),
+                                       "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
         except (FileNotFoundError, OSError):
             self.p = None
+
+    def lines(self) -> int:
+        self.f.flush()
+        try:
+            return sum(1 for _ in open(self.f.name))
+        except OSError:
+            return 0
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_stop(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.p is None:
@@ -101,21 +130,26 @@ class ClockSampler:
         self.f.flush()
         rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
         os.unlink(self.f.name)
-        sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        samples = []
         for r in rows:
             try:
-                sm.append(float(r[1]))
-                mx = float(r[2])
+                ts = time.mktime(time.strptime(r[0].strip().split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + r[0].strip().split(".")[1]) if "." in r[0] else 0.0
+                samples.append((ts, float(r[2]), float(r[3]),
+                                {n for n, v in zip(names, r[6:10]) if v.strip().lower() == "active"}))
             except (ValueError, IndexError):
                 continue
-            for name, v in zip(names, r[5:9]):
-                if v.strip().lower() == "active":
-                    reasons.add(name)
-        if not sm:
+        if not samples or self.t0 is None or self.t1 is None:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [x for x in samples if self.t0 <= x[0] <= self.t1]
+        if not inside:   # timed region shorter than the sampling period: nearest samples
+            mid = 0.5 * (self.t0 + self.t1)
+            inside = sorted(samples, key=lambda x: abs(x[0] - mid))[:2]
+        return {"sm_mhz": float(np.median([x[1] for x in inside])),
+                "sm_max_mhz": inside[-1][2],
+                "reasons": sorted(set().union(*[x[3] for x in inside])),
+                "samples": len(inside)}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -125,7 +159,7 @@ def build_state(w, device):
     import looped_transformer_decode_b200 as lla
 
     cfg = lla.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
-    append = w.encode_tokens < w.B * w.n          # decode-time append: one new row per sequence
+    append = w.encode_tokens <= w.B               # decode-time append: one new row per sequence
     n_cap = w.n + 1 if append else w.n
     layers = []
     for layer in range(w.layers):
@@ -160,7 +194,11 @@ def run_step(lla, w, st, events=None):
             if events is not None:
                 events[1].append(_event())
     for L in st["layers"]:
+        if events is not None:
+            events[2].append(_event())
         lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
+        if events is not None:
+            events[3].append(_event())
 
 
 def _event():
@@ -233,32 +271,52 @@ def run_gpu(args):
     import looped_transformer_decode_b200 as lla
 
     w = synth.WORKLOADS[args.workload]
+    if args.encode_tokens:
+        w = dataclasses.replace(w, encode_tokens=args.encode_tokens)
     st = build_state(w, device)
     for _ in range(max(args.warmup, 3)):
         run_step(lla, w, st)
     barrier_sync(dist_on)
-
+    # the clock sampler starts before more warm-up steps, so its first samples
+    # exist by the time the timed region begins (all ranks take the same steps)
     clocks = ClockSampler(local) if rank == 0 else None
-    ev_pairs = ([], [])
+    t_w = time.time()
+    while True:
+        run_step(lla, w, st)
+        torch.cuda.synchronize()
+        done = 1.0 if (clocks is None or clocks.lines() >= 2 or time.time() - t_w > 5.0) else 0.0
+        if dist_on:
+            flag = torch.tensor([done], device=device)
+            dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+            done = float(flag)
+        if done:
+            break
+
+    ev_pairs = ([], [], [], [])
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier_sync(dist_on)
+    if clocks:
+        clocks.mark_start()
     start.record()
     for _ in range(args.steps):
         run_step(lla, w, st, ev_pairs)
     stop.record()
     barrier_sync(dist_on)
+    if clocks:
+        clocks.mark_stop()
     ms = start.elapsed_time(stop)
     clk = clocks.stop() if clocks else None
-    dec_ms = [a.elapsed_time(b) for a, b in zip(*ev_pairs)]
+    dec_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[0], ev_pairs[1])]
+    enc_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[2], ev_pairs[3])]
     status = lla.decode_status(st["ws"])
     if status:
         raise RuntimeError(f"decode reported device status bits {status}")
     if dist_on:
-        tt = torch.tensor([ms, float(np.mean(dec_ms))], device=device)
+        tt = torch.tensor([ms, float(np.mean(dec_ms)), float(np.mean(enc_ms))], device=device)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, dec_avg = float(tt[0]), float(tt[1])
+        ms, dec_avg, enc_avg = float(tt[0]), float(tt[1]), float(tt[2])
     else:
-        dec_avg = float(np.mean(dec_ms))
+        dec_avg, enc_avg = float(np.mean(dec_ms)), float(np.mean(enc_ms))
 
     per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, w.n)
                       + w.layers * encode_bytes(w, w.encode_tokens))
@@ -266,7 +324,15 @@ def run_gpu(args):
     value = world * per_step_bytes / (ms_step * 1e-3) / 1e9
     ctx_tokens = world * len(w.loops) * w.layers * w.B * w.n / (ms_step * 1e-3)
     peak, peak_kind = peaks()
-    achieved = decode_bytes(w, w.n) / (dec_avg * 1e-3) / 1e9
+    # the roofline is reported for the kernel that takes most of the step: decode
+    # (prep + partial + combine per call) or, for prefill-sized encodes, the encode
+    dec_total = len(w.loops) * w.layers * dec_avg
+    enc_total = w.layers * enc_avg
+    if enc_total > dec_total:
+        unit_bytes, unit_ms, kname = encode_bytes(w, w.encode_tokens), enc_avg, "lla_encode"
+    else:
+        unit_bytes, unit_ms, kname = decode_bytes(w, w.n), dec_avg, "lla_decode_attn (prep + partial + combine)"
+    achieved = unit_bytes / (unit_ms * 1e-3) / 1e9
 
     e2e = None
     if not args.no_e2e:
@@ -287,12 +353,15 @@ def run_gpu(args):
                          "of latents per loop pass)"},
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
-        "roofline": {"bound": "hbm", "kernel": "lla_decode_attn (partial + combine)",
+        "roofline": {"bound": "hbm", "kernel": kname,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC.get(w.name),
+                     "frac": round(achieved / peak, 4),
+                     "traffic": NCU_TRAFFIC.get(w.name) if not args.encode_tokens else None,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "call_us": round(unit_ms * 1e3, 2),
+                     "algorithmic_bytes_per_call": unit_bytes,
                      "decode_call_us": round(dec_avg * 1e3, 2),
-                     "algorithmic_bytes_per_call": decode_bytes(w, w.n)},
+                     "encode_call_us": round(enc_avg * 1e3, 2)},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": e2e,
         "clocks": clk,
