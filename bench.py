@@ -32,8 +32,6 @@ import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = synth.WORKLOAD_ORDER[1]
 METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop step"
-# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu capture
-# summarised in profiles/decode_tc_perhead4x_B8_n4096.md; drop an entry when the kernel changes.
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of the
 # current kernels (profiles/); a workload without a capture of the current code reports null.
 NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 277.10e6,
@@ -54,6 +52,9 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--encode-tokens", type=int, default=0,
                    help="override the workload's tokens encoded per step (profiling aid)")
+    p.add_argument("--evict", default="",
+                   help="SINK,WINDOW: decode over a sink + window retention budget of the "
+                        "history (eviction composed with the latent cache)")
     return p.parse_args()
 
 
@@ -185,7 +186,35 @@ def build_state(w, device):
             "slot": slot, "out": out, "n_cap": n_cap}
 
 
+def apply_eviction(lla, w, st, sink: int, window: int) -> int:
+    """Keep a sink + window budget of each sequence's n-token history.
+
+    Slot bookkeeping of lla_evict_slot: the kept tokens' positions are written at
+    their slots and ctx_len becomes the budget; the new token of each step is
+    appended at the slot lla_evict_append gives position n.  Returns the number of
+    attended history tokens.
+    """
+    import torch
+
+    keep = list(range(min(sink, w.n))) + list(range(max(sink, w.n - window), w.n))
+    slots = [lla.evict_slot(sink, window, p) for p in keep]
+    n_cap = st["n_cap"]
+    for L in st["layers"]:
+        pos = L["positions"]
+        pos[:, torch.tensor(slots, device=pos.device)] = torch.tensor(keep, dtype=pos.dtype,
+                                                                      device=pos.device)
+        L["ctx_len"].fill_(len(keep))
+    if w.encode_tokens <= w.B:                    # decode-time append into the ring
+        pos_new = torch.full((w.B,), w.n, dtype=torch.int32, device=st["slot"].device)
+        pos_tab = st["layers"][0]["positions"].clone()
+        ctx_tab = st["layers"][0]["ctx_len"].clone()
+        st["slot"] = lla.evict_append(w.B, n_cap, sink, window, pos_new, pos_tab, ctx_tab)
+    return len(keep)
+
+
 def run_step(lla, w, st, events=None):
+    if st.get("flush") is not None:
+        st["flush"].add_(1)                       # working set below L2: evict it first
     for t in w.loops:
         for L in st["layers"]:
             if events is not None:
@@ -276,6 +305,17 @@ def run_gpu(args):
     if args.encode_tokens:
         w = dataclasses.replace(w, encode_tokens=args.encode_tokens)
     st = build_state(w, device)
+    n_ctx = w.n
+    evict = None
+    if args.evict:
+        evict = tuple(int(v) for v in args.evict.split(","))
+        n_ctx = apply_eviction(lla, w, st, *evict)
+    l2_note = (f"inputs larger than L2 ({decode_bytes(w, n_ctx) * w.layers / 1e6:.0f} MB "
+               "of latents per loop pass)")
+    if decode_bytes(w, n_ctx) * w.layers < 256e6:
+        st["flush"] = torch.zeros(96 * 2**20, dtype=torch.int32, device=device)   # 384 MB
+        l2_note = ("L2 flushed each step by a 384 MB write (inside the step time; the "
+                   "decode call times exclude it)")
     for _ in range(max(args.warmup, 3)):
         run_step(lla, w, st)
     barrier_sync(dist_on)
@@ -320,11 +360,11 @@ def run_gpu(args):
     else:
         dec_avg, enc_avg = float(np.mean(dec_ms)), float(np.mean(enc_ms))
 
-    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, w.n)
+    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, n_ctx)
                       + w.layers * encode_bytes(w, w.encode_tokens))
     ms_step = ms / args.steps
     value = world * per_step_bytes / (ms_step * 1e-3) / 1e9
-    ctx_tokens = world * len(w.loops) * w.layers * w.B * w.n / (ms_step * 1e-3)
+    ctx_tokens = world * len(w.loops) * w.layers * w.B * n_ctx / (ms_step * 1e-3)
     peak, peak_kind = peaks()
     # the roofline is reported for the kernel that takes most of the step: decode
     # (prep + partial + combine per call) or, for prefill-sized encodes, the encode
@@ -333,12 +373,12 @@ def run_gpu(args):
     if enc_total > dec_total:
         unit_bytes, unit_ms, kname = encode_bytes(w, w.encode_tokens), enc_avg, "lla_encode"
     else:
-        unit_bytes, unit_ms, kname = decode_bytes(w, w.n), dec_avg, "lla_decode_attn (prep + partial + combine)"
+        unit_bytes, unit_ms, kname = decode_bytes(w, n_ctx), dec_avg, "lla_decode_attn (prep + partial + combine)"
     achieved = unit_bytes / (unit_ms * 1e-3) / 1e9
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(lla, w, st, args, dist_on, world)
+        e2e = run_e2e(lla, w, st, args, dist_on, world, n_ctx)
 
     launches_per_step = (len(w.loops) * w.layers * lla.decode_launches(st["cfg"], w.B, st["n_cap"])
                          + w.layers)
@@ -351,14 +391,15 @@ def run_gpu(args):
                    "r_v": w.r_v, "mode": "per_head" if w.mode == synth.MODE_PER_HEAD else "lla_2d",
                    "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
                    "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2 ({decode_bytes(w, w.n) * w.layers / 1e6:.0f} MB "
-                         "of latents per loop pass)"},
+                   "evict": list(evict) if evict else None, "attended_context": n_ctx,
+                   "l2": l2_note},
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
         "roofline": {"bound": "hbm", "kernel": kname,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": NCU_TRAFFIC.get(w.name) if not args.encode_tokens else None,
+                     "traffic": (NCU_TRAFFIC.get(w.name)
+                                 if not (args.encode_tokens or args.evict) else None),
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "call_us": round(unit_ms * 1e3, 2),
                      "algorithmic_bytes_per_call": unit_bytes,
@@ -377,7 +418,7 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_e2e(lla, w, st, args, dist_on, world):
+def run_e2e(lla, w, st, args, dist_on, world, n_ctx):
     """Same step with inputs copied from pinned host memory and the output read back."""
     import torch
 
@@ -425,7 +466,7 @@ def run_e2e(lla, w, st, args, dist_on, world):
         tt = torch.tensor([ms], device=st["out"].device)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt[0])
-    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, w.n)
+    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, n_ctx)
                       + w.layers * encode_bytes(w, w.encode_tokens))
     return {"value": round(world * per_step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),

@@ -251,6 +251,40 @@ int lla_decode_attn_noalloc(const lla_cfg* cfg, const void* packed, const void* 
  */
 int lla_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap);
 
+/* ------------------------------------------------------------------------ */
+/*
+ * Eviction composed with the latent cache: a sink + window retention budget
+ * (close reading §四.10, Table 9: 4 sink tokens + a 256-token window; Appendix J:
+ * a 1024-token budget).  The first `sink` history tokens and the `window` most
+ * recent ones are kept, each at its own position.  A sequence's cache rows then
+ * act as sink + window slots: history position p < sink lives in slot p, and
+ * p >= sink in slot sink + (p - sink) mod window, overwriting the position that
+ * just left the window.  Each slot's positions entry holds its token's position
+ * and the decode reads slots [0, ctx_len) with ctx_len = min(n, sink + window);
+ * attention over a set does not depend on slot order, so lla_decode_attn is
+ * used unchanged.  No data moves when a token is evicted.
+ */
+
+/* Slot (row within its sequence) of history position pos; host only, exact.
+ * Returns -1 when sink < 0, window < 1 or pos < 0. */
+int64_t lla_evict_slot(int32_t sink, int32_t window, int64_t pos);
+
+/*
+ * Decode-time append under eviction, one new history token per sequence:
+ *   pos        device int32 [B]: history position of each sequence's new token
+ *              (its index in the history: the previous ctx_len when nothing was
+ *              evicted yet); pos < 0 leaves the sequence untouched and writes
+ *              slot -1 (lla_encode then skips it).
+ *   slot       device int64 [B] (out): flat cache row b * n_cap + slot for lla_encode.
+ *   positions  device int32 [B][n_cap] (in/out): the slot's entry is set to pos.
+ *   ctx_len    device int32 [B] (out): min(pos + 1, sink + window).
+ * Requires B >= 0, n_cap >= 1, sink >= 0, window >= 1 and sink + window <= n_cap
+ * (LLA_ERR_INVALID otherwise); pointers 8-byte (slot) or 4-byte aligned.
+ * Enqueued on `stream`; B == 0 is a no-op.
+ */
+int lla_evict_append(int32_t B, int32_t n_cap, int32_t sink, int32_t window, const int32_t* pos,
+                     int64_t* slot, int32_t* positions, int32_t* ctx_len, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

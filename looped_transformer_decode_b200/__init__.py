@@ -19,6 +19,7 @@ __all__ = [
     "Cfg", "LLAError", "MODE_PER_HEAD", "MODE_2D", "ratio", "cache_bytes", "codec_pack",
     "rope_table", "encode", "decode_workspace", "decode_attn", "decode_status", "lib",
     "decode_launches", "STATUS_POSITION_RANGE", "STATUS_CTX_RANGE", "STATUS_SLOT_RANGE",
+    "evict_slot", "evict_append",
 ]
 
 
@@ -151,3 +152,23 @@ def decode_attn(cfg: Cfg, packed, rope, t: int, ctx_len, q, k_self, v_self, posi
         _ptr(out, torch.float32, "out", (B, H, d)), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream()))
     return out
+
+
+def evict_slot(sink: int, window: int, pos: int) -> int:
+    """Slot (row within its sequence) of history position ``pos`` under sink + window eviction."""
+    return int(lib.lla_evict_slot(sink, window, pos))
+
+
+def evict_append(B: int, n_cap: int, sink: int, window: int, pos, positions, ctx_len, slot=None):
+    """Slots for one new history token per sequence under sink + window eviction.
+
+    ``pos`` int32 [B] device: history position of each new token.  Updates ``positions``
+    [B, n_cap] and ``ctx_len`` [B] in place; returns the flat slots int64 [B] for encode.
+    """
+    if slot is None:
+        slot = torch.empty((B,), dtype=torch.int64, device=pos.device)
+    check(lib.lla_evict_append(B, n_cap, sink, window, _ptr(pos, torch.int32, "pos", (B,)),
+                               _ptr(slot, torch.int64, "slot", (B,)),
+                               _ptr(positions, torch.int32, "positions", (B, n_cap)),
+                               _ptr(ctx_len, torch.int32, "ctx_len", (B,)), _stream()))
+    return slot

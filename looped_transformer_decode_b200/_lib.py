@@ -77,6 +77,8 @@ SIGNATURES = {
     "lla_decode_launches": (ctypes.c_int, [_CFG, _I32, _I32]),
     "lla_decode_attn_noalloc": (ctypes.c_int, [_CFG, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P,
                                                _P, _P, _P, _P, _P, _P, _P, _P]),
+    "lla_evict_slot": (_I64, [_I32, _I32, _I64]),
+    "lla_evict_append": (ctypes.c_int, [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(lib, _name)

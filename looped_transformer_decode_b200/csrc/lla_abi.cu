@@ -362,4 +362,28 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   return ok();
 }
 
+
+int64_t lla_evict_slot(int32_t sink, int32_t window, int64_t pos) {
+  return lla::evict_slot(sink, window, pos);
+}
+
+int lla_evict_append(int32_t B, int32_t n_cap, int32_t sink, int32_t window, const int32_t* pos,
+                     int64_t* slot, int32_t* positions, int32_t* ctx_len, void* stream) {
+  if (B < 0 || n_cap < 1) return fail(LLA_ERR_INVALID, "lla_evict_append: B must be >= 0 and n_cap >= 1");
+  if (sink < 0 || window < 1) return fail(LLA_ERR_INVALID, "lla_evict_append: need sink >= 0 and window >= 1");
+  if ((int64_t)sink + window > n_cap)
+    return fail(LLA_ERR_INVALID, "lla_evict_append: sink + window = %lld exceeds n_cap = %d",
+                (long long)sink + window, n_cap);
+  if (B == 0) return ok();
+  if (!pos || !slot || !positions || !ctx_len)
+    return fail(LLA_ERR_INVALID, "lla_evict_append: NULL pointer argument");
+  if ((reinterpret_cast<uintptr_t>(slot) & 7u) || (reinterpret_cast<uintptr_t>(pos) & 3u) ||
+      (reinterpret_cast<uintptr_t>(positions) & 3u) || (reinterpret_cast<uintptr_t>(ctx_len) & 3u))
+    return fail(LLA_ERR_INVALID, "lla_evict_append: misaligned pointer");
+  cudaError_t ce = lla::launch_evict_append(B, n_cap, sink, window, pos, slot, positions, ctx_len,
+                                            static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce, "lla_evict_append launch");
+  return ok();
+}
+
 }  // extern "C"

@@ -71,6 +71,12 @@ cudaError_t launch_encode_tc(const lla_cfg& c, const PackedLayout& L, const char
                              const int64_t* slot, int64_t n_slots, __nv_bfloat16* ck,
                              __nv_bfloat16* cv, int32_t* status, cudaStream_t s);
 
+// Eviction (sink + window slots over the latent cache).
+int64_t evict_slot(int32_t sink, int32_t window, int64_t pos);
+cudaError_t launch_evict_append(int B, int n_cap, int sink, int window, const int32_t* pos,
+                                int64_t* slot, int32_t* positions, int32_t* ctx_len,
+                                cudaStream_t s);
+
 struct DecodeArgs {
   int T, H, d, r_k, r_v, mode;
   float kappa;           // sm_scale * log2(e): scores are kept in base-2 units

@@ -357,3 +357,35 @@ def svd_codec(cfg: Cfg, calib_k: np.ndarray, calib_v: np.ndarray) -> Codec:
     mv, Wv, _ = svd_init(calib_v.reshape(N, -1), cfg.r_v)
     return Codec(Wk, Wv, loop_slices(Wk, cfg.T, cfg.d, cfg.H), loop_slices(Wv, cfg.T, cfg.d, cfg.H),
                  mk, mv)
+
+
+# --------------------------------------------------------------------------
+# Eviction composed with LLA ([CR] §四.10, Table 9 and Appendix J)
+# --------------------------------------------------------------------------
+
+def evict_keep(n: int, sink: int, window: int) -> np.ndarray:
+    """History indices kept by a sink + window retention budget out of n tokens.
+
+    [CR] §四.10 evaluates LLA under a 260-token budget, 4 sink tokens plus a
+    256-token window, and Appendix J under a 1024-token one: the first ``sink``
+    tokens and the ``window`` most recent ones stay.  Each keeps its own position
+    (eviction drops tokens, it does not renumber the survivors; the page does not
+    say, and this is the plain reading).
+    """
+    if n <= sink + window:
+        return np.arange(n)
+    return np.concatenate([np.arange(sink), np.arange(n - window, n)])
+
+
+def decode_attention_evicted(q, k_self, v_self, c_k, c_v, W_up_k_t, W_up_v_t, mu_k_t, mu_v_t,
+                             pos_hist, q_pos, base, sink, window, scale=None):
+    """decode_attention over the tokens that sink + window keeps.
+
+    c_k, c_v and pos_hist cover the whole history (n rows); the in-flight token
+    is attended as always.
+    """
+    keep = evict_keep(len(pos_hist), sink, window)
+    pos_hist = np.asarray(pos_hist)
+    return decode_attention(q, k_self, v_self, np.asarray(c_k)[keep], np.asarray(c_v)[keep],
+                            W_up_k_t, W_up_v_t, mu_k_t, mu_v_t, pos_hist[keep], q_pos, base,
+                            scale)
