@@ -260,14 +260,19 @@ size_t lla_decode_workspace_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap) 
   if (check_cfg(cfg) || B < 0 || n_cap < 0) return 0;
   ok();
   SplitPlan p = split_plan(*cfg, B, n_cap);
-  return kWsHeader + align_up(partials_bytes(*cfg, B, p.splits), 256) + p.ops_bytes;
+  return kWsHeader + align_up(partials_bytes(*cfg, B, p.splits), 256) + align_up(p.ops_bytes, 256) +
+         (p.tensor_cores ? align_up(((size_t)B * cfg->H + 1) * 4, 256) : 0);
 }
 
 int lla_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap) {
   if (check_cfg(cfg) || B < 0 || n_cap < 0) return -1;
   if (B == 0) return 0;
   if (n_cap == 0) return 1;
-  return split_plan(*cfg, B, n_cap).tensor_cores ? 3 : 2;
+  // tensor cores: prep + partials + combine, the combine fused into the partials
+  // when each per-head group has a single split; CUDA cores: partials + combine
+  const SplitPlan sp = split_plan(*cfg, B, n_cap);
+  if (!sp.tensor_cores) return 2;
+  return (cfg->mode == LLA_MODE_PER_HEAD && sp.splits == 1) ? 2 : 3;
 }
 
 int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_table,
@@ -297,7 +302,9 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
     }
   }
   SplitPlan plan = split_plan(*cfg, B, n_cap);
-  size_t need = kWsHeader + align_up(partials_bytes(*cfg, B, plan.splits), 256) + plan.ops_bytes;
+  const size_t ops_at = kWsHeader + align_up(partials_bytes(*cfg, B, plan.splits), 256);
+  const size_t counters_at = ops_at + align_up(plan.ops_bytes, 256);
+  size_t need = counters_at + (plan.tensor_cores ? align_up(((size_t)B * cfg->H + 1) * 4, 256) : 0);
   if (ws_bytes < need)
     return fail(LLA_ERR_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
 
@@ -347,16 +354,14 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   a.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
   a.S = plan.splits;
   a.tiles_per_split = plan.tiles_per_split;
-  a.ops = plan.tensor_cores
-              ? static_cast<unsigned char*>(ws) + kWsHeader +
-                    align_up(partials_bytes(*cfg, B, plan.splits), 256)
-              : nullptr;
+  a.ops = plan.tensor_cores ? static_cast<unsigned char*>(ws) + ops_at : nullptr;
+  a.counters = plan.tensor_cores
+                   ? reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + counters_at)
+                   : nullptr;
   int launches = 0;
   cudaError_t ce = cudaErrorNotSupported;
-  if (plan.tensor_cores && plan.splits > 0) {
+  if (plan.tensor_cores && plan.splits > 0)
     ce = launch_decode_tc(*cfg, a, static_cast<cudaStream_t>(stream));
-    if (ce == cudaSuccess) ce = launch_combine(a, static_cast<cudaStream_t>(stream));
-  }
   if (ce == cudaErrorNotSupported) ce = launch_decode(a, static_cast<cudaStream_t>(stream), &launches);
   if (ce != cudaSuccess) return cuda_fail(ce, "lla_decode_attn launch");
   return ok();

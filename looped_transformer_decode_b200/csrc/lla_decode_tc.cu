@@ -66,6 +66,19 @@ struct TcParams {
   // LLA-2D kernel: B-operand buffers, P rows (N of the V MMA), 128-row blocks of r_v
   int nbuf_b, n_p, m_v;
   int poll;                                  // per-head hand-offs poll instead of suspending
+  // fused split combine (per-head kernel): the CTA that finishes a group's last split
+  // merges the splits, adds the in-flight token and up-projects with W_up,v
+  const float* q;                            // [B][H][d]
+  const float* k_self;
+  const float* v_self;
+  const float* wupv_t;                       // [H][r_v][d] at loop t
+  const float* muv_t;                        // [H][d]
+  float* out;                                // [B][H][d]
+  float kappa;
+  int d;
+  uint32_t* counters;                        // [B * H] finished splits per group, then CTAs done
+  uint32_t comb_off;                         // smem: olat [r_v], split weights [64], reductions
+  int fuse_combine;                          // 1: the combine is done here (one split per group)
   uint32_t p_buf_bytes;
   const float2* rope;    // [rope_max_pos][d/2]
   const int32_t* ctx_len;
@@ -290,10 +303,15 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
     const float* __restrict__ q, const int32_t* __restrict__ q_pos, const float2* __restrict__ rope,
     int rope_max_pos, const float* __restrict__ wupk_t, const float* __restrict__ muk_t, float kappa,
     int H, int r_k, int K_pad, unsigned char* __restrict__ ops_b,
-    unsigned char* __restrict__ ops_bias, int32_t* status) {
+    unsigned char* __restrict__ ops_bias, int32_t* status, uint32_t* counters) {
   constexpr int HALF = D / 2;
   __shared__ float2 qc[HALF];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  // the fused combine's counters start every call at zero (this kernel runs first)
+  if (counters && blockIdx.z == 0 && tid == 0) {
+    counters[(size_t)b * H + h] = 0u;
+    if (h == 0 && b == 0) counters[(size_t)gridDim.y * H] = 0u;
+  }
   int qp = q_pos[b];
   if (qp < 0 || qp >= rope_max_pos) {
     if (tid == 0 && h == 0 && blockIdx.z == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
@@ -354,7 +372,78 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
 // is rescaled to a new reference maximum.
 constexpr float kRescaleLog2 = 8.f;
 
-template <int D, int G>
+// Split combine of head (b, h), run by the 128 threads of one warpgroup (named
+// barrier `bar`): merge the S split partials (m, l, sum p c_v) at a common
+// maximum, add the in-flight token (its score q . k_self needs no rotation: both
+// sit at q_pos), and o = W_up,v (sum p c_v) / l + (sum_hist p / l) mu_v + (p_self / l)
+// v_self.  Same arithmetic as decode_combine_kernel.  Partials written by other
+// CTAs are read past L1 (ld.global.cg).
+__device__ void combine_head(const TcParams& p, int b, int h, unsigned char* scratch, int tid,
+                             uint32_t bar) {
+  float* olat = reinterpret_cast<float*>(scratch);   // [r_v]
+  float* wts = olat + 256;                            // [64] split weights
+  float* red = wts + 64;                              // [8]
+  const int lane = tid & 31, w = tid >> 5;
+  const size_t bh = (size_t)b * p.H + h;
+  const int stride = 2 + p.r_v;
+  const float* parts = p.partials + bh * p.S * stride;
+  float m_s = -INFINITY, dot = 0.f;
+  if (tid < p.S) m_s = __ldcg(parts + (size_t)tid * stride);
+  for (int i = tid; i < p.d; i += 128) dot = fmaf(p.q[bh * p.d + i], p.k_self[bh * p.d + i], dot);
+  const float mx = warp_max_f(m_s), ds = warp_sum_f(dot);
+  if (lane == 0) {
+    red[w] = mx;
+    red[4 + w] = ds;
+  }
+  named_barrier(bar, 128);
+  const float M_hist = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float s_self = p.kappa * ((red[4] + red[5]) + (red[6] + red[7]));
+  const float M = fmaxf(M_hist, s_self);
+  if (tid < p.S) wts[tid] = exp2f(m_s - M);
+  named_barrier(bar, 128);
+  // loads are issued in batches of 8 or 16 before they are used: from L2 under load
+  // each round trip is long, and only a warpgroup runs this
+  float l_hist = 0.f;
+  for (int s0 = 0; s0 < p.S; s0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = s0 + e < p.S ? __ldcg(parts + (size_t)(s0 + e) * stride + 1) : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) l_hist = fmaf(v[e], s0 + e < p.S ? wts[s0 + e] : 0.f, l_hist);
+  }
+  const float w_self = exp2f(s_self - M);
+  const float inv = 1.f / (l_hist + w_self);
+  for (int m = tid; m < p.r_v; m += 128) {
+    float acc = 0.f;
+    for (int s0 = 0; s0 < p.S; s0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        v[e] = s0 + e < p.S ? __ldcg(parts + (size_t)(s0 + e) * stride + 2 + m) : 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(v[e], s0 + e < p.S ? wts[s0 + e] : 0.f, acc);
+    }
+    olat[m] = acc * inv;
+  }
+  named_barrier(bar, 128);
+  if (tid < p.d) {
+    // W_up,v,t,h packed transposed ([r_v][d]): the loads of consecutive threads coalesce
+    const float* Wt = p.wupv_t + (size_t)h * p.d * p.r_v + tid;
+    float y = 0.f;
+    for (int m0 = 0; m0 < p.r_v; m0 += 16) {
+      float wv[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) wv[e] = m0 + e < p.r_v ? Wt[(size_t)(m0 + e) * p.d] : 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) y = fmaf(wv[e], m0 + e < p.r_v ? olat[m0 + e] : 0.f, y);
+    }
+    p.out[bh * p.d + tid] = y + (l_hist * inv) * p.muv_t[(size_t)h * p.d + tid] +
+                            (w_self * inv) * p.v_self[bh * p.d + tid];
+  }
+  named_barrier(bar, 128);   // scratch is reused by the next head
+}
+
+template <int D, int G, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
@@ -832,6 +921,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.partials[((bh0 + g) * p.S + r.s) * (2 + p.r_v) + m] = m == 0 ? -INFINITY : 0.f;
         }
       }
+      if constexpr (FUSE) if (wgi == 0) {
+        // ---- fused combine: the CTA that finishes a group's last split merges it
+        uint32_t* flag = reinterpret_cast<uint32_t*>(sm + p.comb_off) + 328;
+        __threadfence();                       // this split's partials are visible first
+        named_barrier(2, 128);
+        if (row == 0)
+          flag[0] = atomicAdd(&p.counters[(size_t)r.b * p.HG + r.hg], 1u) == (uint32_t)(p.S - 1);
+        named_barrier(2, 128);
+        if (flag[0]) {
+          __threadfence();
+          for (int g = 0; g < G; ++g) combine_head(p, r.b, r.hg * G + g, sm + p.comb_off, row, 2);
+        }
+      }
     }
   }
 
@@ -841,7 +943,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+  if (threadIdx.x == 0) {
+    if (*abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+    if constexpr (FUSE) {
+      // with the combine fused in, the last CTA to finish publishes this call's status
+      // bits (word 1) and clears word 0; otherwise the combine pass does it
+      __threadfence();
+      if (atomicAdd(&p.counters[(size_t)p.B * p.H], 1u) == gridDim.x - 1) {
+        __threadfence();
+        p.status[1] = atomicExch(&p.status[0], 0);
+      }
+    }
+  }
 }
 
 // LLA-2D: every head reads the same latent row (close reading §二.6), so a work
@@ -1369,6 +1482,8 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst, int nst_v) {
   o += 2 * G * 8 * kTile * 2;
   p.sbuf_off = o;
   o += 2 * (kEpiWG - 1) * G * kTile * 4;
+  p.comb_off = o;                    // fused combine: olat [256], split weights [64], red [8], flag
+  o += (256 + 64 + 8 + 4) * 4;
   p.red_off = o;
   o = al(o + G * 4 * 4, 16);
   p.ctx_off = o;
@@ -1552,7 +1667,8 @@ bool tc_enabled() {
 template <int D, int G, bool SHARED>
 cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
                         uint32_t smem, int grid, cudaStream_t s) {
-  auto kern = SHARED ? decode_tc2d_kernel<D, G> : decode_tc_kernel<D, G>;
+  auto kern = SHARED ? decode_tc2d_kernel<D, G>
+                     : (p.fuse_combine ? decode_tc_kernel<D, G, true> : decode_tc_kernel<D, G, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, SHARED ? kThreads2 : kThreads, smem, s>>>(mk, mv, p);
@@ -1581,7 +1697,7 @@ cudaError_t launch_prep(const DecodeArgs& a, const TcParams& p, cudaStream_t s) 
 #define LLA_PREP(DD)                                                                          \
   decode_prep_kernel<DD><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, \
                                               a.muk_t, a.kappa, a.H, a.r_k, p.K_pad, ob, obias, \
-                                              a.status)
+                                              a.status, a.counters)
   switch (a.d) {
     case 32: LLA_PREP(32); break;
     case 64: LLA_PREP(64); break;
@@ -1660,6 +1776,21 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.positions = a.positions;
   p.status = a.status;
   p.partials = a.partials;
+  p.q = a.q;
+  p.k_self = a.k_self;
+  p.v_self = a.v_self;
+  p.wupv_t = a.wupv_t;
+  p.muv_t = a.muv_t;
+  p.out = a.out;
+  p.kappa = a.kappa;
+  p.d = a.d;
+  p.counters = a.counters;
+  if (!a.counters) return cudaErrorNotSupported;
+  // Fused only when a group has one split: its combine then runs right after the
+  // group's own tiles on the same CTA.  A cross-CTA merge inside this streaming
+  // kernel waits on L2 round trips behind the latent traffic (measured: far slower
+  // than the separate pass), so several splits keep the combine pass.
+  p.fuse_combine = (!pl.shared && pl.S == 1) ? 1 : 0;
   if (!a.ops) return cudaErrorNotSupported;
   p.ops_b = a.ops;
   p.ops_bias = a.ops + (size_t)a.B * a.H * p.b_head_bytes;
@@ -1682,13 +1813,16 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   cudaError_t pe = launch_prep(a, p, s);
   if (pe != cudaSuccess) return pe;
   const int grid = p.n_items < sms ? p.n_items : sms;
+  cudaError_t e;
   switch (a.d) {
-    case 32: return launch_tc_d<32>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
-    case 64: return launch_tc_d<64>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
-    case 96: return launch_tc_d<96>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
-    case 128: return launch_tc_d<128>(pl.G, pl.shared, mk, mv, p, smem, grid, s);
+    case 32: e = launch_tc_d<32>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+    case 64: e = launch_tc_d<64>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+    case 96: e = launch_tc_d<96>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+    case 128: e = launch_tc_d<128>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
     default: return cudaErrorNotSupported;
   }
+  if (e == cudaSuccess && !p.fuse_combine) e = launch_combine(a, s);
+  return e;
 }
 
 }  // namespace lla
