@@ -272,7 +272,7 @@ int lla_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap) {
   // when each per-head group has a single split; CUDA cores: partials + combine
   const SplitPlan sp = split_plan(*cfg, B, n_cap);
   if (!sp.tensor_cores) return 2;
-  return (cfg->mode == LLA_MODE_PER_HEAD && sp.splits == 1) ? 2 : 3;
+  return sp.splits == 1 ? 2 : 3;
 }
 
 int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_table,

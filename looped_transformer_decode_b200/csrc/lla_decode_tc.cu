@@ -978,7 +978,7 @@ constexpr int kEpiWarps2 = kEpiThreads2 / 32;
 constexpr int kThreads2 = 64 + kEpiThreads2 + 64;
 constexpr int kVProdWarp2 = 2 + kEpiWarps2, kVMmaWarp2 = 3 + kEpiWarps2;
 
-template <int D, int HP>
+template <int D, int HP, bool FUSE>
 __global__ void __launch_bounds__(kThreads2, 1)
     decode_tc2d_kernel(const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
@@ -1401,6 +1401,15 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const size_t bh = (size_t)r.b * p.H + r.hg * HP + wgi;
         for (int m = row; m < 2 + p.r_v; m += 128)
           p.partials[(bh * p.S + r.s) * (2 + p.r_v) + m] = m == 0 ? -INFINITY : 0.f;
+        named_barrier(2 + wgi, 128);
+      }
+      if constexpr (FUSE) if (fin) {
+        // one split per group: finalize head wgi right away.  Scratch: this
+        // warpgroup's slice of the partial-exchange buffer of the parity no tile
+        // touches until every warpgroup has passed the next tile's barrier.
+        unsigned char* scratch = reinterpret_cast<unsigned char*>(
+            sbuf + ((((it - 1u) & 1u) * HP + wgi) * kEpiWG2) * kTile);
+        combine_head(p, r.b, r.hg * HP + wgi, scratch, row, 2 + wgi);
       }
     }
   }
@@ -1411,7 +1420,17 @@ __global__ void __launch_bounds__(kThreads2, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+  if (threadIdx.x == 0) {
+    if (*abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+    if constexpr (FUSE) {
+      // the last CTA to finish publishes this call's status bits (word 1)
+      __threadfence();
+      if (atomicAdd(&p.counters[(size_t)p.B * p.H], 1u) == gridDim.x - 1) {
+        __threadfence();
+        p.status[1] = atomicExch(&p.status[0], 0);
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -1667,7 +1686,7 @@ bool tc_enabled() {
 template <int D, int G, bool SHARED>
 cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
                         uint32_t smem, int grid, cudaStream_t s) {
-  auto kern = SHARED ? decode_tc2d_kernel<D, G>
+  auto kern = SHARED ? (p.fuse_combine ? decode_tc2d_kernel<D, G, true> : decode_tc2d_kernel<D, G, false>)
                      : (p.fuse_combine ? decode_tc_kernel<D, G, true> : decode_tc_kernel<D, G, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1790,7 +1809,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   // group's own tiles on the same CTA.  A cross-CTA merge inside this streaming
   // kernel waits on L2 round trips behind the latent traffic (measured: far slower
   // than the separate pass), so several splits keep the combine pass.
-  p.fuse_combine = (!pl.shared && pl.S == 1) ? 1 : 0;
+  p.fuse_combine = pl.S == 1 ? 1 : 0;
   if (!a.ops) return cudaErrorNotSupported;
   p.ops_b = a.ops;
   p.ops_bias = a.ops + (size_t)a.B * a.H * p.b_head_bytes;
