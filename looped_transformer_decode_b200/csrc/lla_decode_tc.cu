@@ -28,9 +28,11 @@
 // LLA_STATUS_TIMEOUT, drains its in-flight copies, frees TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <vector>
 
 #include "lla_internal.cuh"
 #include "lla_sm100.cuh"
@@ -1652,23 +1654,40 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   pl.nst = best_nst;
   pl.nst_v = best_nst_v;
   pl.nacc = best_nacc;
-  // Context splits: balance tiles over a 148-SM grid of persistent CTAs.
+  // Context splits: the split count S minimises the busiest CTA's cost over a
+  // 148-SM grid of persistent CTAs, where items are dealt round-robin and each
+  // item costs its tiles plus a fixed start/finish charge (operand hand-over, the
+  // V-accumulator drain and the partial write, about 1.6 tiles of time measured on
+  // the per-head 4x workload); more than one split also pays the combine pass.
   const int n_tiles = (n_cap + kTile - 1) / kTile;
   const long long units = (long long)B * (c.H / pl.G);
   const int grid = 148;
-  double best_eff = -1.0;
+  constexpr double kItemCost = 1.6, kCombineCost = 0.5;   // in tiles
+  const int forced_s = env_int("LLA_TC_SPLITS", 0);
+  int s_max = (int)std::max<long long>(1, (4 * grid + units - 1) / units);
+  s_max = std::min(std::min(s_max, kMaxSplits), n_tiles);
+  double best_cost = 1e300;
   int best_s = 1;
-  for (int S = 1; S <= kMaxSplits && S <= n_tiles; ++S) {
+  for (int S = forced_s > 0 ? forced_s : 1; S <= (forced_s > 0 ? forced_s : s_max); ++S) {
     const int tpi = (n_tiles + S - 1) / S;
     const int s_eff = (n_tiles + tpi - 1) / tpi;
     const long long items = units * s_eff;
-    const long long per_cta = (items + grid - 1) / grid * tpi;
-    const double eff = (double)units * n_tiles / ((double)grid * per_cta);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    double worst = 0.0;
+    if (items > grid) {
+      std::vector<double> cta(grid, 0.0);
+      for (long long it = 0; it < items; ++it) {
+        const int sp = (int)(it % s_eff);
+        cta[it % grid] += std::min(tpi, n_tiles - sp * tpi) + kItemCost;
+      }
+      for (double v : cta) worst = std::max(worst, v);
+    } else {
+      worst = tpi + kItemCost;
+    }
+    const double cost = worst + (s_eff > 1 ? kCombineCost : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
       best_s = s_eff;
     }
-    if (eff >= 0.93) break;
   }
   pl.tps = (n_tiles + best_s - 1) / best_s;
   pl.S = (n_tiles + pl.tps - 1) / pl.tps;
