@@ -389,3 +389,93 @@ def decode_attention_evicted(q, k_self, v_self, c_k, c_v, W_up_k_t, W_up_v_t, mu
     return decode_attention(q, k_self, v_self, np.asarray(c_k)[keep], np.asarray(c_v)[keep],
                             W_up_k_t, W_up_v_t, mu_k_t, mu_v_t, pos_hist[keep], q_pos, base,
                             scale)
+
+
+# --------------------------------------------------------------------------
+# Full-memory fast path ([CR] §四.9, Table 5 row "full-memory fast path" and the
+# paragraph after the table; §二.3 for where RoPE sits)
+# --------------------------------------------------------------------------
+
+def full_memory_kv(c_k, c_v, W_up_k_t, W_up_v_t, mu_k_t, mu_v_t, positions, base,
+                   round_bf16=True):
+    """Loop-t K and V of a history as a full cache keeps them.
+
+    [CR] §四.9: the full-memory fast path stores the complete rebuilt K/V (so it
+    gives up the cache saving) instead of rebuilding on every read.  Per [CR]
+    §二.3 the codec works on pre-RoPE K and the model rotates the rebuilt key at
+    its position before caching it, so the stored key is
+        K_j = RoPE(c_k,j W_up,k,t^T + mu_k,t, positions[j])
+    and the stored value V_j = c_v,j W_up,v,t^T + mu_v,t.  The cache number
+    format is bf16 (2 bytes per scalar, as in the Table 5 teacher row), so both
+    are rounded once; ``round_bf16=False`` keeps float64.
+    Returns (K [n, d], V [n, d]).
+    """
+    K = rope(reconstruct(c_k, W_up_k_t, mu_k_t), np.asarray(positions), base)
+    V = reconstruct(c_v, W_up_v_t, mu_v_t)
+    if round_bf16:
+        return bf16_round(K), bf16_round(V)
+    return K, V
+
+
+def decode_attention_full(q, k_self, v_self, K_rot, V, q_pos, base, scale=None):
+    """Ordinary decode attention over a full cache whose keys are already rotated.
+
+    q, k_self, v_self: [d] pre-RoPE (the in-flight token, loop t); K_rot, V: [n, d].
+      s_j    = scale * RoPE(q, q_pos) . K_rot,j
+      s_self = scale * RoPE(q, q_pos) . RoPE(k_self, q_pos)
+      p      = softmax over the n history scores and s_self
+      out    = sum_j p_j V_j + p_self v_self
+    """
+    q = np.asarray(q, np.float64)
+    d = q.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    K_rot = np.asarray(K_rot, np.float64).reshape(-1, d)
+    V = np.asarray(V, np.float64).reshape(-1, d)
+    q_rot = rope(q, q_pos, base)
+    scores = np.empty(K_rot.shape[0] + 1)
+    for j in range(K_rot.shape[0]):
+        scores[j] = scale * float(np.dot(q_rot, K_rot[j]))
+    scores[-1] = scale * float(np.dot(q_rot, rope(np.asarray(k_self, np.float64), q_pos, base)))
+    w = np.exp(scores - scores.max())
+    w /= w.sum()
+    return w[:-1] @ V + w[-1] * np.asarray(v_self, np.float64)
+
+
+def full_cache(cfg: Cfg, codec: Codec, t: int, c_k, c_v, positions, ctx_len, round_bf16=True):
+    """The full-memory cache of loop t in the library's layout, head-major.
+
+    c_k, c_v, positions: latent-cache layout ([B, n_cap, H, r] per head, [B, n_cap, r]
+    LLA-2D; positions [B, n_cap]).  Returns (K [B, H, n_cap, d], V [B, H, n_cap, d])
+    with rows j < ctx_len[b] filled by ``full_memory_kv`` and the rest zero.
+    """
+    B, n_cap = np.asarray(positions).shape
+    K = np.zeros((B, cfg.H, n_cap, cfg.d))
+    V = np.zeros((B, cfg.H, n_cap, cfg.d))
+    for b in range(B):
+        n = int(ctx_len[b])
+        for h in range(cfg.H):
+            if cfg.mode == MODE_PER_HEAD:
+                ck, cv = np.asarray(c_k[b, :n, h]), np.asarray(c_v[b, :n, h])
+            else:
+                ck, cv = np.asarray(c_k[b, :n]), np.asarray(c_v[b, :n])
+            K[b, h, :n], V[b, h, :n] = full_memory_kv(
+                ck, cv, w_up_t(cfg, codec.W_up_k, t, h), w_up_t(cfg, codec.W_up_v, t, h),
+                mu_t(cfg, codec.mu_k, t, h), mu_t(cfg, codec.mu_v, t, h),
+                np.asarray(positions[b, :n]), cfg.rope_base, round_bf16)
+    return K, V
+
+
+def decode_attn_full_cache(cfg: Cfg, q, k_self, v_self, K_full, V_full, q_pos, ctx_len,
+                           scale=None):
+    """``decode_attention_full`` for a batch.  q, k_self, v_self: [B, H, d];
+    K_full, V_full: [B, H, n_cap, d]; q_pos, ctx_len: [B].  Returns [B, H, d]."""
+    q = np.asarray(q, np.float64)
+    B, H, d = q.shape
+    out = np.zeros((B, H, d))
+    for b in range(B):
+        n = int(ctx_len[b])
+        for h in range(H):
+            out[b, h] = decode_attention_full(q[b, h], k_self[b, h], v_self[b, h],
+                                              K_full[b, h, :n], V_full[b, h, :n],
+                                              int(q_pos[b]), cfg.rope_base, scale)
+    return out
