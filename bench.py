@@ -38,6 +38,8 @@ NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 277.77e6,
                "lla2d_T4_H16_d128_r64_128_B512_n4096": 1013.46e6,
                # encode (the dominant kernel): a 32768-token capture scaled by 16 tokens-wise
                "deeploop_32x_T32_H8_d96_r64_128_B16_n32768": 55.24e9}
+# The same for the full-memory fast path (dominant kernel: full_decode_kernel).
+NCU_TRAFFIC_FULL = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 272.19e6}
 
 
 def parse():
@@ -52,6 +54,10 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--encode-tokens", type=int, default=0,
                    help="override the workload's tokens encoded per step (profiling aid)")
+    p.add_argument("--path", default="latent", choices=["latent", "full"],
+                   help="latent: decode over the latent cache (rebuild on read); full: the "
+                        "full-memory fast path (K/V rebuilt once per token into a full bf16 "
+                        "cache per loop, ordinary attention)")
     p.add_argument("--evict", default="",
                    help="SINK,WINDOW: decode over a sink + window retention budget of the "
                         "history (eviction composed with the latent cache)")
@@ -68,6 +74,20 @@ def decode_bytes(w, n_ctx: int) -> int:
     weights = w.H * w.d * (w.r_k + w.r_v) * 4 + 2 * w.H * w.d * 4
     io = 4 * w.B * w.H * w.d * 4
     return lat + pos + weights + io
+
+
+def full_decode_bytes(w, n_ctx: int) -> int:
+    """Algorithmic HBM bytes of one full-memory decode call: bf16 K and V rows of the
+    attended history plus the per-head inputs and output."""
+    return w.B * w.H * n_ctx * 2 * w.d * 2 + 4 * w.B * w.H * w.d * 4 + 2 * w.B * 4
+
+
+def full_rebuild_bytes(w, n_rows: int) -> int:
+    """Bytes of rebuilding n_rows cache rows at one loop: latents and positions in,
+    W_up and mu, bf16 K/V rows out."""
+    L = w.H if w.mode == synth.MODE_PER_HEAD else 1
+    return (n_rows * (L * (w.r_k + w.r_v) * 2 + 4 + 8) + w.H * w.d * (w.r_k + w.r_v + 2) * 4
+            + n_rows * w.H * 2 * w.d * 2)
 
 
 def encode_bytes(w, n_tok: int) -> int:
@@ -212,7 +232,62 @@ def apply_eviction(lla, w, st, sink: int, window: int) -> int:
     return len(keep)
 
 
+def build_full(lla, w, st, device):
+    """Full-memory fast path: rebuild every history row once into a bf16 K/V cache per
+    (layer, loop).  Returns the rebuild time of one (layer, loop) cache in ms."""
+    import torch
+
+    need = w.layers * len(w.loops) * 2 * lla.full_kv_bytes(st["cfg"], w.B, st["n_cap"])
+    free, _ = torch.cuda.mem_get_info(device)
+    if need > 0.85 * free:
+        raise SystemExit(f"full-memory path needs {need / 2**30:.1f} GiB of full K/V caches for "
+                         f"{w.layers} layers x {len(w.loops)} loops; {free / 2**30:.1f} GiB free")
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rebuild_ms = []
+    for L in st["layers"]:
+        L["full"] = {}
+        for t in w.loops:
+            kf, vf = lla.full_cache_alloc(st["cfg"], w.B, st["n_cap"], device)
+            s.record()
+            lla.full_rebuild(st["cfg"], L["packed"], st["rope"], t, L["positions"], L["c_k"],
+                             L["c_v"], kf, vf)
+            e.record()
+            torch.cuda.synchronize()
+            rebuild_ms.append(s.elapsed_time(e))
+            L["full"][t] = (kf, vf)
+    st["fws"] = lla.full_decode_workspace(st["cfg"], w.B, st["n_cap"], device)
+    return float(np.median(rebuild_ms))
+
+
+def run_step_full(lla, w, st, events=None):
+    """One step of the fast path: decode every loop over its full cache, then encode
+    the new tokens and rebuild their rows into every loop's cache."""
+    if st.get("flush") is not None:
+        st["flush"].add_(1)
+    for t in w.loops:
+        for L in st["layers"]:
+            if events is not None:
+                events[0].append(_event())
+            kf, vf = L["full"][t]
+            lla.full_decode_attn(st["cfg"], st["rope"], L["ctx_len"], L["q"], L["k_self"],
+                                 L["v_self"], L["q_pos"], kf, vf, out=st["out"], ws=st["fws"])
+            if events is not None:
+                events[1].append(_event())
+    for L in st["layers"]:
+        if events is not None:
+            events[2].append(_event())
+        lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
+        for t in w.loops:
+            kf, vf = L["full"][t]
+            lla.full_rebuild(st["cfg"], L["packed"], st["rope"], t, L["positions"], L["c_k"],
+                             L["c_v"], kf, vf, slot=st["slot"])
+        if events is not None:
+            events[3].append(_event())
+
+
 def run_step(lla, w, st, events=None):
+    if st.get("full_path"):
+        return run_step_full(lla, w, st, events)
     if st.get("flush") is not None:
         st["flush"].add_(1)                       # working set below L2: evict it first
     for t in w.loops:
@@ -310,9 +385,17 @@ def run_gpu(args):
     if args.evict:
         evict = tuple(int(v) for v in args.evict.split(","))
         n_ctx = apply_eviction(lla, w, st, *evict)
-    l2_note = (f"inputs larger than L2 ({decode_bytes(w, n_ctx) * w.layers / 1e6:.0f} MB "
-               "of latents per loop pass)")
-    if decode_bytes(w, n_ctx) * w.layers < 256e6:
+    full = args.path == "full"
+    rebuild_once_ms = None
+    if full:
+        if evict:
+            raise SystemExit("--path full does not combine with --evict")
+        rebuild_once_ms = build_full(lla, w, st, device)
+        st["full_path"] = True
+    dec_bytes = full_decode_bytes if full else decode_bytes
+    l2_note = (f"inputs larger than L2 ({dec_bytes(w, n_ctx) * w.layers / 1e6:.0f} MB "
+               f"of {'full K/V' if full else 'latents'} per loop pass)")
+    if dec_bytes(w, n_ctx) * w.layers < 256e6:
         st["flush"] = torch.zeros(96 * 2**20, dtype=torch.int32, device=device)   # 384 MB
         l2_note = ("L2 flushed each step by a 384 MB write (inside the step time; the "
                    "decode call times exclude it)")
@@ -350,7 +433,7 @@ def run_gpu(args):
     clk = clocks.stop() if clocks else None
     dec_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[0], ev_pairs[1])]
     enc_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[2], ev_pairs[3])]
-    status = lla.decode_status(st["ws"])
+    status = lla.decode_status(st["fws"] if full else st["ws"])
     if status:
         raise RuntimeError(f"decode reported device status bits {status}")
     if dist_on:
@@ -360,8 +443,10 @@ def run_gpu(args):
     else:
         dec_avg, enc_avg = float(np.mean(dec_ms)), float(np.mean(enc_ms))
 
-    per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, n_ctx)
-                      + w.layers * encode_bytes(w, w.encode_tokens))
+    append_bytes = encode_bytes(w, w.encode_tokens)
+    if full:
+        append_bytes += len(w.loops) * full_rebuild_bytes(w, st["slot"].numel())
+    per_step_bytes = (len(w.loops) * w.layers * dec_bytes(w, n_ctx) + w.layers * append_bytes)
     ms_step = ms / args.steps
     value = world * per_step_bytes / (ms_step * 1e-3) / 1e9
     ctx_tokens = world * len(w.loops) * w.layers * w.B * n_ctx / (ms_step * 1e-3)
@@ -371,17 +456,26 @@ def run_gpu(args):
     dec_total = len(w.loops) * w.layers * dec_avg
     enc_total = w.layers * enc_avg
     if enc_total > dec_total:
-        unit_bytes, unit_ms, kname = encode_bytes(w, w.encode_tokens), enc_avg, "lla_encode"
+        unit_bytes, unit_ms = append_bytes, enc_avg
+        kname = "lla_encode + lla_full_rebuild" if full else "lla_encode"
     else:
-        unit_bytes, unit_ms, kname = decode_bytes(w, n_ctx), dec_avg, "lla_decode_attn (prep + partial + combine)"
+        unit_bytes, unit_ms = dec_bytes(w, n_ctx), dec_avg
+        kname = ("lla_full_decode_attn (full_decode_kernel [+ combine])" if full
+                 else "lla_decode_attn (prep + partial + combine)")
     achieved = unit_bytes / (unit_ms * 1e-3) / 1e9
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not full:
         e2e = run_e2e(lla, w, st, args, dist_on, world, n_ctx)
 
-    launches_per_step = (len(w.loops) * w.layers * lla.decode_launches(st["cfg"], w.B, st["n_cap"])
-                         + w.layers)
+    if full:
+        launches_per_step = (len(w.loops) * w.layers
+                             * lla.full_decode_launches(st["cfg"], w.B, st["n_cap"])
+                             + w.layers * (1 + len(w.loops)))
+    else:
+        launches_per_step = (len(w.loops) * w.layers
+                             * lla.decode_launches(st["cfg"], w.B, st["n_cap"]) + w.layers)
+    traffic_table = NCU_TRAFFIC_FULL if full else NCU_TRAFFIC
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
@@ -392,13 +486,13 @@ def run_gpu(args):
                    "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
                    "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
                    "evict": list(evict) if evict else None, "attended_context": n_ctx,
-                   "l2": l2_note},
+                   "path": args.path, "l2": l2_note},
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
         "roofline": {"bound": "hbm", "kernel": kname,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": (NCU_TRAFFIC.get(w.name)
+                     "traffic": (traffic_table.get(w.name)
                                  if not (args.encode_tokens or args.evict) else None),
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "call_us": round(unit_ms * 1e3, 2),
@@ -409,13 +503,48 @@ def run_gpu(args):
         "e2e": e2e,
         "clocks": clk,
     }
+    if full:
+        line["config"]["full_cache_gib"] = round(
+            w.layers * len(w.loops) * 2 * lla.full_kv_bytes(st["cfg"], w.B, st["n_cap"]) / 2**30, 2)
+        line["config"]["rebuild_once_ms_per_layer_loop"] = round(rebuild_once_ms, 3)
+        line["e2e_note"] = "end-to-end line measured on the latent path (the default)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = (cpu_baseline_full(w, args.cpu_seconds) if full
+                                else cpu_baseline_sample(w, args.cpu_seconds))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def cpu_baseline_full(w, seconds: float):
+    """Time the float64 oracle's full-memory attention on (b, h) pairs at full context
+    (bf16-valued K/V rows drawn at random: the cost does not depend on the values)."""
+    import oracle as O
+
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    g = synth.rng(w.seed + 7)
+    K = O.bf16_round(g.standard_normal((w.n, w.d)))
+    V = O.bf16_round(g.standard_normal((w.n, w.d)))
+    q, ks, vs = (g.standard_normal(w.d) for _ in range(3))
+    pairs = 0
+    t0 = time.perf_counter()
+    while True:
+        O.decode_attention_full(q, ks, vs, K, V, w.n, 10000.0)
+        pairs += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and pairs >= 2:
+            break
+    per_pair = full_decode_bytes(w, w.n) / (w.B * w.H)
+    return {"value": pairs * per_pair / el / 1e9, "unit": "GB/s", "cores": int(threads),
+            "kind": "oracle", "seconds": round(el, 2),
+            "sample": f"{pairs} (b,h) pairs x {w.n} context tokens, float64 NumPy "
+                      f"decode_attention_full; bytes scaled as the GPU path's per pair"}
 
 
 def run_e2e(lla, w, st, args, dist_on, world, n_ctx):

@@ -285,6 +285,68 @@ int64_t lla_evict_slot(int32_t sink, int32_t window, int64_t pos);
 int lla_evict_append(int32_t B, int32_t n_cap, int32_t sink, int32_t window, const int32_t* pos,
                      int64_t* slot, int32_t* positions, int32_t* ctx_len, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* Full-memory fast path: rebuild once, then ordinary attention.              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The close reading ("Looped Latent Attention: 跨循环 KV 压缩精读", §四.9, Table 5
+ * and the paragraph after it) contrasts the latent store (keep only latents,
+ * rebuild on every read) with a full-memory fast path that keeps the complete
+ * rebuilt K/V, giving up the cache saving for speed.  Per §二.3 the codec works
+ * on pre-RoPE K and the model rotates the rebuilt key at its position before it
+ * is cached, so the full cache holds rotated keys.
+ *
+ * Full cache of one loop t: k_full and v_full, each device bf16 [B][H][n_cap][d]
+ * (head-major: one (sequence, head) history is a contiguous run of rows).
+ */
+
+/* Bytes of one of k_full / v_full for (cfg, B, n_cap); 0 if the arguments are invalid. */
+size_t lla_full_kv_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap);
+
+/*
+ * Rebuild rows of the loop-t full cache from the latent cache:
+ *   k_full[b][h][j] = bf16(RoPE(c_k[b][j](h) W_up,k,t,h^T + mu_k,t,h, positions[b][j]))
+ *   v_full[b][h][j] = bf16(c_v[b][j](h) W_up,v,t,h^T + mu_v,t,h)
+ * for each row b * n_cap + j listed in slot[0 .. n_rows) (device int64), or for
+ * rows 0 .. n_rows-1 when slot is NULL (n_rows <= B * n_cap; B * n_cap rebuilds the
+ * whole cache once).  c_k, c_v and positions are laid out as for lla_decode_attn;
+ * packed and rope_table as for lla_decode_attn.  status (optional device int32)
+ * collects LLA_STATUS_SLOT_RANGE (a slot outside [0, B * n_cap): skipped) and
+ * LLA_STATUS_POSITION_RANGE (a position outside the table: clamped).  Runs on the
+ * CUDA cores; it is a once-per-token conversion, not a per-step cost.
+ */
+int lla_full_rebuild(const lla_cfg* cfg, const void* packed, const void* rope_table,
+                     int32_t rope_max_pos, int32_t t, int32_t B, int32_t n_cap,
+                     const int32_t* positions, const uint16_t* c_k, const uint16_t* c_v,
+                     const int64_t* slot, int64_t n_rows, uint16_t* k_full, uint16_t* v_full,
+                     int32_t* status, void* stream);
+
+/* Workspace bytes for lla_full_decode_attn (zero-filled once before first use; its
+ * first two int32 words are the status words described at lla_decode_workspace_bytes). */
+size_t lla_full_decode_workspace_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap);
+
+/* Kernel launches one lla_full_decode_attn call makes (1 or 2), or -1 if invalid. */
+int lla_full_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap);
+
+/*
+ * out[b][h] = ordinary decode attention over the full cache plus the in-flight token:
+ *   s_j   = sm_scale * RoPE(q, q_pos[b]) . k_full[b][h][j]   (j < ctx_len[b])
+ *   s_self = sm_scale * RoPE(q, q_pos[b]) . RoPE(k_self, q_pos[b])
+ *   out   = sum_j p_j v_full[b][h][j] + p_self v_self,  p = softmax(s, s_self)
+ *   q, k_self, v_self  device fp32 [B][H][d], pre-RoPE; q_pos, ctx_len device int32 [B]
+ *   k_full, v_full     device bf16 [B][H][n_cap][d] (may be NULL when n_cap == 0)
+ *   out                device fp32 [B][H][d]
+ * The cfg's codec fields (T, r_k, r_v, mode) are not used.  B * H * n_cap must stay
+ * below 2^31 rows (LLA_ERR_UNSUPPORTED otherwise).  Device-side range problems set
+ * LLA_STATUS_POSITION_RANGE / LLA_STATUS_CTX_RANGE in the workspace status word.
+ */
+int lla_full_decode_attn(const lla_cfg* cfg, const void* rope_table, int32_t rope_max_pos,
+                         int32_t B, int32_t n_cap, const int32_t* ctx_len, const float* q,
+                         const float* k_self, const float* v_self, const int32_t* q_pos,
+                         const uint16_t* k_full, const uint16_t* v_full, float* out, void* ws,
+                         size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,8 @@ __all__ = [
     "Cfg", "LLAError", "MODE_PER_HEAD", "MODE_2D", "ratio", "cache_bytes", "codec_pack",
     "rope_table", "encode", "decode_workspace", "decode_attn", "decode_status", "lib",
     "decode_launches", "STATUS_POSITION_RANGE", "STATUS_CTX_RANGE", "STATUS_SLOT_RANGE",
-    "evict_slot", "evict_append",
+    "evict_slot", "evict_append", "full_kv_bytes", "full_cache_alloc", "full_rebuild",
+    "full_decode_workspace", "full_decode_launches", "full_decode_attn",
 ]
 
 
@@ -172,3 +173,78 @@ def evict_append(B: int, n_cap: int, sink: int, window: int, pos, positions, ctx
                                _ptr(positions, torch.int32, "positions", (B, n_cap)),
                                _ptr(ctx_len, torch.int32, "ctx_len", (B,)), _stream()))
     return slot
+
+
+# ---------------------------------------------------------------- full-memory fast path
+
+def full_kv_bytes(cfg: Cfg, B: int, n_cap: int) -> int:
+    """Bytes of one loop's full K (or V) cache, bf16 [B, H, n_cap, d]."""
+    return int(lib.lla_full_kv_bytes(ctypes.byref(cfg.c()), B, n_cap))
+
+
+def full_cache_alloc(cfg: Cfg, B: int, n_cap: int, device="cuda"):
+    """Empty full K and V caches of one loop, bf16 [B, H, n_cap, d] each."""
+    shape = (B, cfg.H, n_cap, cfg.d_head)
+    return (torch.zeros(shape, dtype=torch.bfloat16, device=device),
+            torch.zeros(shape, dtype=torch.bfloat16, device=device))
+
+
+def full_rebuild(cfg: Cfg, packed, rope, t: int, positions, c_k, c_v, k_full, v_full,
+                 slot=None, n_rows=None, status=None):
+    """Rebuild rows of the loop-t full cache (in place) from the latent cache.
+
+    ``slot`` int64 [n] lists rows b * n_cap + j; without it rows 0 .. n_rows-1 (default:
+    every row) are rebuilt.
+    """
+    c = cfg.c()
+    B, n_cap = positions.shape
+    fs = (B, cfg.H, n_cap, cfg.d_head)
+    if slot is not None:
+        n_rows = slot.shape[0]
+        sp = _ptr(slot, torch.int64, "slot", (n_rows,))
+    else:
+        n_rows = B * n_cap if n_rows is None else n_rows
+        sp = None
+    st = _ptr(status, torch.int32, "status") if status is not None else None
+    check(lib.lla_full_rebuild(
+        ctypes.byref(c), _ptr(packed, torch.uint8, "packed"), _ptr(rope, torch.float32, "rope"),
+        rope.shape[0], t, B, n_cap, _ptr(positions, torch.int32, "positions", (B, n_cap)),
+        _ptr(c_k, torch.bfloat16, "c_k", _cache_shape(cfg, (B, n_cap), cfg.r_k)),
+        _ptr(c_v, torch.bfloat16, "c_v", _cache_shape(cfg, (B, n_cap), cfg.r_v)),
+        sp, n_rows, _ptr(k_full, torch.bfloat16, "k_full", fs),
+        _ptr(v_full, torch.bfloat16, "v_full", fs), st, _stream()))
+
+
+def full_decode_workspace(cfg: Cfg, B: int, n_cap: int, device="cuda"):
+    n = lib.lla_full_decode_workspace_bytes(ctypes.byref(cfg.c()), B, n_cap)
+    if n == 0:
+        raise LLAError(ERR_UNSUPPORTED, last_error())
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def full_decode_launches(cfg: Cfg, B: int, n_cap: int) -> int:
+    return lib.lla_full_decode_launches(ctypes.byref(cfg.c()), B, n_cap)
+
+
+def full_decode_attn(cfg: Cfg, rope, ctx_len, q, k_self, v_self, q_pos, k_full, v_full,
+                     out=None, ws=None):
+    """Ordinary decode attention over the full cache; returns out fp32 [B, H, d]."""
+    c = cfg.c()
+    B, H, d = q.shape
+    n_cap = k_full.shape[2]
+    if H != cfg.H or d != cfg.d_head:
+        raise ValueError("q shape does not match cfg")
+    fs = (B, H, n_cap, d)
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = full_decode_workspace(cfg, B, n_cap, q.device)
+    check(lib.lla_full_decode_attn(
+        ctypes.byref(c), _ptr(rope, torch.float32, "rope"), rope.shape[0], B, n_cap,
+        _ptr(ctx_len, torch.int32, "ctx_len", (B,)), _ptr(q, torch.float32, "q", (B, H, d)),
+        _ptr(k_self, torch.float32, "k_self", (B, H, d)),
+        _ptr(v_self, torch.float32, "v_self", (B, H, d)), _ptr(q_pos, torch.int32, "q_pos", (B,)),
+        _ptr(k_full, torch.bfloat16, "k_full", fs), _ptr(v_full, torch.bfloat16, "v_full", fs),
+        _ptr(out, torch.float32, "out", (B, H, d)), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream()))
+    return out

@@ -79,6 +79,13 @@ SIGNATURES = {
                                                _P, _P, _P, _P, _P, _P, _P, _P]),
     "lla_evict_slot": (_I64, [_I32, _I32, _I64]),
     "lla_evict_append": (ctypes.c_int, [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _P]),
+    "lla_full_kv_bytes": (_SZ, [_CFG, _I32, _I32]),
+    "lla_full_rebuild": (ctypes.c_int, [_CFG, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P,
+                                        _I64, _P, _P, _P, _P]),
+    "lla_full_decode_workspace_bytes": (_SZ, [_CFG, _I32, _I32]),
+    "lla_full_decode_launches": (ctypes.c_int, [_CFG, _I32, _I32]),
+    "lla_full_decode_attn": (ctypes.c_int, [_CFG, _P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P,
+                                            _P, _P, _P, _SZ, _P]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(lib, _name)

@@ -391,4 +391,140 @@ int lla_evict_append(int32_t B, int32_t n_cap, int32_t sink, int32_t window, con
   return ok();
 }
 
+// ---------------------------------------------------------------- full-memory fast path
+
+size_t lla_full_kv_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap) {
+  if (check_cfg(cfg) || B < 0 || n_cap < 0) return 0;
+  return (size_t)B * cfg->H * (size_t)n_cap * cfg->d_head * 2;
+}
+
+int lla_full_rebuild(const lla_cfg* cfg, const void* packed, const void* rope_table,
+                     int32_t rope_max_pos, int32_t t, int32_t B, int32_t n_cap,
+                     const int32_t* positions, const uint16_t* c_k, const uint16_t* c_v,
+                     const int64_t* slot, int64_t n_rows, uint16_t* k_full, uint16_t* v_full,
+                     int32_t* status, void* stream) {
+  int e = check_cfg(cfg);
+  if (e) return e;
+  if (t < 0 || t >= cfg->T) return fail(LLA_ERR_INVALID, "t=%d outside [0, T=%d)", t, cfg->T);
+  if (B < 0 || n_cap < 0 || n_rows < 0)
+    return fail(LLA_ERR_INVALID, "B, n_cap and n_rows must be >= 0");
+  if (rope_max_pos < 1) return fail(LLA_ERR_INVALID, "rope_max_pos must be >= 1");
+  if (!slot && n_rows > (int64_t)B * n_cap)
+    return fail(LLA_ERR_INVALID, "n_rows=%lld above B * n_cap without a slot list",
+                (long long)n_rows);
+  if (n_rows == 0) return ok();
+  const void* ptrs[] = {packed, rope_table, positions, c_k, c_v, k_full, v_full};
+  for (const void* p : ptrs) {
+    if (!p) return fail(LLA_ERR_INVALID, "lla_full_rebuild: NULL pointer argument");
+    if (!aligned16(p)) return fail(LLA_ERR_INVALID, "lla_full_rebuild: pointer not 16-byte aligned");
+  }
+  if (slot && !aligned16(slot)) return fail(LLA_ERR_INVALID, "lla_full_rebuild: slot misaligned");
+  if (status && (reinterpret_cast<uintptr_t>(status) & 3u))
+    return fail(LLA_ERR_INVALID, "lla_full_rebuild: status not 4-byte aligned");
+  PackedLayout L = packed_layout(*cfg);
+  const char* pk = static_cast<const char*>(packed);
+  const size_t d = cfg->d_head, H = cfg->H;
+  FullRebuildArgs a{};
+  a.d = cfg->d_head;
+  a.H = cfg->H;
+  a.r_k = cfg->r_k;
+  a.r_v = cfg->r_v;
+  a.B = B;
+  a.n_cap = n_cap;
+  a.rope_max_pos = rope_max_pos;
+  a.n_rows = n_rows;
+  a.slot = slot;
+  a.positions = positions;
+  a.rope = static_cast<const float2*>(rope_table);
+  a.wupk_t = reinterpret_cast<const float*>(pk + L.wupk) + (size_t)t * H * d * cfg->r_k;
+  a.wupv_t = reinterpret_cast<const float*>(pk + L.wupv) + (size_t)t * H * d * cfg->r_v;
+  a.muk_t = reinterpret_cast<const float*>(pk + L.muk) + (size_t)t * H * d;
+  a.muv_t = reinterpret_cast<const float*>(pk + L.muv) + (size_t)t * H * d;
+  a.ck = reinterpret_cast<const __nv_bfloat16*>(c_k);
+  a.cv = reinterpret_cast<const __nv_bfloat16*>(c_v);
+  const bool per_head = cfg->mode == LLA_MODE_PER_HEAD;
+  a.lat_tok_k = per_head ? (long long)H * cfg->r_k : cfg->r_k;
+  a.lat_tok_v = per_head ? (long long)H * cfg->r_v : cfg->r_v;
+  a.lat_head_k = per_head ? cfg->r_k : 0;
+  a.lat_head_v = per_head ? cfg->r_v : 0;
+  a.k_full = reinterpret_cast<__nv_bfloat16*>(k_full);
+  a.v_full = reinterpret_cast<__nv_bfloat16*>(v_full);
+  a.status = status;
+  cudaError_t ce = launch_full_rebuild(a, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce, "lla_full_rebuild launch");
+  return ok();
+}
+
+size_t lla_full_decode_workspace_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap) {
+  if (check_cfg(cfg) || B < 0 || n_cap < 0) return 0;
+  FullPlan pl = full_plan(*cfg, B, n_cap);
+  const size_t parts = pl.S > 1 ? (size_t)B * cfg->H * pl.S * (cfg->d_head + 2) * 4 : 0;
+  return kWsHeader + align_up(parts, 256);
+}
+
+int lla_full_decode_launches(const lla_cfg* cfg, int32_t B, int32_t n_cap) {
+  if (check_cfg(cfg) || B < 0 || n_cap < 0) return -1;
+  if (B == 0) return 0;
+  return full_plan(*cfg, B, n_cap).S > 1 ? 2 : 1;
+}
+
+int lla_full_decode_attn(const lla_cfg* cfg, const void* rope_table, int32_t rope_max_pos,
+                         int32_t B, int32_t n_cap, const int32_t* ctx_len, const float* q,
+                         const float* k_self, const float* v_self, const int32_t* q_pos,
+                         const uint16_t* k_full, const uint16_t* v_full, float* out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  int e = check_cfg(cfg);
+  if (e) return e;
+  if (B < 0 || n_cap < 0) return fail(LLA_ERR_INVALID, "B and n_cap must be >= 0");
+  if (rope_max_pos < 1) return fail(LLA_ERR_INVALID, "rope_max_pos must be >= 1");
+  if ((long long)B * cfg->H * (long long)n_cap > (long long)INT32_MAX)
+    return fail(LLA_ERR_UNSUPPORTED, "B * H * n_cap above 2^31-1 cache rows");
+  if (B == 0) return ok();
+  const void* ptrs[] = {rope_table, ctx_len, q, k_self, v_self, q_pos, out, ws};
+  for (const void* p : ptrs) {
+    if (!p) return fail(LLA_ERR_INVALID, "lla_full_decode_attn: NULL pointer argument");
+    if (!aligned16(p))
+      return fail(LLA_ERR_INVALID, "lla_full_decode_attn: pointer not 16-byte aligned");
+  }
+  if (n_cap > 0) {
+    const void* hist[] = {k_full, v_full};
+    for (const void* p : hist) {
+      if (!p) return fail(LLA_ERR_INVALID, "lla_full_decode_attn: NULL cache pointer");
+      if (!aligned16(p)) return fail(LLA_ERR_INVALID, "lla_full_decode_attn: cache misaligned");
+    }
+  }
+  const size_t need = lla_full_decode_workspace_bytes(cfg, B, n_cap);
+  if (ws_bytes < need)
+    return fail(LLA_ERR_TOO_SMALL, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  FullPlan pl = full_plan(*cfg, B, n_cap);
+  FullDecodeParams p{};
+  p.B = B;
+  p.H = cfg->H;
+  p.n_cap = n_cap;
+  p.d = cfg->d_head;
+  p.S = pl.S;
+  p.tps = pl.tps;
+  p.n_items = (int)pl.n_items;
+  p.rope_max_pos = rope_max_pos;
+  p.fuse = pl.S == 1 ? 1 : 0;
+  const float scale = cfg->sm_scale > 0.f ? cfg->sm_scale : 1.0f / std::sqrt((float)cfg->d_head);
+  p.kappa = (float)((double)scale * 1.4426950408889634);  // log2(e): base-2 scores
+  p.q = q;
+  p.k_self = k_self;
+  p.v_self = v_self;
+  p.q_pos = q_pos;
+  p.ctx_len = ctx_len;
+  p.rope = static_cast<const float2*>(rope_table);
+  p.out = out;
+  p.status = static_cast<int32_t*>(ws);
+  p.counter = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16);
+  p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeader);
+  // with no history the tensor maps are never read; any aligned address encodes them
+  const void* kb = n_cap > 0 ? static_cast<const void*>(k_full) : ws;
+  const void* vb = n_cap > 0 ? static_cast<const void*>(v_full) : ws;
+  cudaError_t ce = launch_full_decode(p, kb, vb, pl.grid, static_cast<cudaStream_t>(stream));
+  if (ce != cudaSuccess) return cuda_fail(ce, "lla_full_decode_attn launch");
+  return ok();
+}
+
 }  // extern "C"

@@ -113,6 +113,48 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 bool decode_tc_plan(const lla_cfg& c, int B, int n_cap, int* S, int* tps, size_t* ops_bytes);
 cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t s);
 
+// Full-memory fast path: the loop-t K/V rebuilt once into a full bf16 cache
+// [B][H][n_cap][d] (keys rotated), and ordinary decode attention over it.
+struct FullRebuildArgs {
+  int d, H, r_k, r_v, B, n_cap, rope_max_pos;
+  long long n_rows;
+  const int64_t* slot;             // [n_rows] rows b * n_cap + j, or null: rows 0 .. n_rows-1
+  const int32_t* positions;        // [B][n_cap]
+  const float2* rope;              // [rope_max_pos][d/2]
+  const float* wupk_t;             // [H][d][r_k] at loop t
+  const float* wupv_t;             // [H][r_v][d]
+  const float* muk_t;              // [H][d]
+  const float* muv_t;
+  const __nv_bfloat16* ck;
+  const __nv_bfloat16* cv;
+  long long lat_tok_k, lat_tok_v, lat_head_k, lat_head_v;
+  __nv_bfloat16* k_full;
+  __nv_bfloat16* v_full;
+  int32_t* status;                 // optional
+};
+struct FullDecodeParams {
+  int B, H, n_cap, d, S, tps, n_items, rope_max_pos, fuse;
+  float kappa;
+  const float* q;
+  const float* k_self;
+  const float* v_self;
+  const int32_t* q_pos;
+  const int32_t* ctx_len;
+  const float2* rope;
+  float* out;
+  float* partials;                 // [B][H][S][2 + d] when S > 1
+  int32_t* status;                 // ws words [0], [1]
+  uint32_t* counter;               // ws word [4]: CTAs finished in this call
+};
+struct FullPlan {
+  int S = 1, tps = 1, grid = 1, grid_max = 148;
+  long long n_items = 0;
+};
+FullPlan full_plan(const lla_cfg& c, int B, int n_cap);
+cudaError_t launch_full_rebuild(const FullRebuildArgs& a, cudaStream_t s);
+cudaError_t launch_full_decode(const FullDecodeParams& p, const void* k_full, const void* v_full,
+                               int grid, cudaStream_t s);
+
 // Record `fmt` as the calling thread's lla_last_error() message; returns `code`.
 int set_error(int code, const char* fmt, ...);
 
