@@ -78,7 +78,7 @@ struct TcParams {
   float* out;                                // [B][H][d]
   float kappa;
   int d;
-  uint32_t* counters;                        // [B * H] finished splits per group, then CTAs done
+  uint32_t* counters;                        // word B * H: CTAs done (fused combine); rest unused
   uint32_t comb_off;                         // smem: olat [r_v], split weights [64], reductions
   int fuse_combine;                          // 1: the combine is done here (one split per group)
   uint32_t p_buf_bytes;
@@ -309,11 +309,10 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
   constexpr int HALF = D / 2;
   __shared__ float2 qc[HALF];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  // the fused combine's counters start every call at zero (this kernel runs first)
-  if (counters && blockIdx.z == 0 && tid == 0) {
-    counters[(size_t)b * H + h] = 0u;
-    if (h == 0 && b == 0) counters[(size_t)gridDim.y * H] = 0u;
-  }
+  // the CTA counter of the fused-combine kernels starts every call at zero (this
+  // kernel runs first)
+  if (counters && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0)
+    counters[(size_t)gridDim.y * H] = 0u;
   int qp = q_pos[b];
   if (qp < 0 || qp >= rope_max_pos) {
     if (tid == 0 && h == 0 && blockIdx.z == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
@@ -924,17 +923,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if constexpr (FUSE) if (wgi == 0) {
-        // ---- fused combine: the CTA that finishes a group's last split merges it
-        uint32_t* flag = reinterpret_cast<uint32_t*>(sm + p.comb_off) + 328;
-        __threadfence();                       // this split's partials are visible first
+        // ---- fused combine: the group has one split, computed right here
+        __threadfence();
         named_barrier(2, 128);
-        if (row == 0)
-          flag[0] = atomicAdd(&p.counters[(size_t)r.b * p.HG + r.hg], 1u) == (uint32_t)(p.S - 1);
-        named_barrier(2, 128);
-        if (flag[0]) {
-          __threadfence();
-          for (int g = 0; g < G; ++g) combine_head(p, r.b, r.hg * G + g, sm + p.comb_off, row, 2);
-        }
+        for (int g = 0; g < G; ++g) combine_head(p, r.b, r.hg * G + g, sm + p.comb_off, row, 2);
       }
     }
   }

@@ -102,7 +102,7 @@ struct DecodeArgs {
   float* partials;       // [B][H][S][2 + r_v]
   int S, tiles_per_split;
   unsigned char* ops;    // per-(b, h) MMA operand images (tensor-core path), or null
-  uint32_t* counters;    // [B * H + 1] fused-combine counters (tensor-core path), or null
+  uint32_t* counters;    // [B * H + 1]; word B * H counts finished CTAs (fused combine), or null
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
