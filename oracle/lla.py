@@ -479,3 +479,97 @@ def decode_attn_full_cache(cfg: Cfg, q, k_self, v_self, K_full, V_full, q_pos, c
                                               K_full[b, h, :n], V_full[b, h, :n],
                                               int(q_pos[b]), cfg.rope_base, scale)
     return out
+
+
+# --------------------------------------------------------------------------
+# Decoupled RoPE ([CR] §四.10, Appendix J and Tables 13-14): a NoPE content path
+# absorbed into the query plus an explicit rotary branch of d_rope dims
+# --------------------------------------------------------------------------
+
+def rope_partial(x, pos, base: float, d_rope: int) -> np.ndarray:
+    """RoPE on the first d_rope dims of x only, as a rotary vector of its own width
+    (split-half pairs (i, i + d_rope/2) at angle pos * base^(-2i/d_rope)); the other
+    d - d_rope dims pass through unrotated.  d_rope = d is the full RoPE of ``rope``.
+
+    Reading: [CR] App. J names a NoPE content path and an explicit rotary branch of
+    d_rope = 64 or 32 dims without saying which dims rotate; the plain reading is
+    the usual partial-rotary layout (leading dims, their own frequency ladder).
+    """
+    x = np.asarray(x, np.float64)
+    if d_rope == 0:
+        return x.copy()
+    return np.concatenate([rope(x[..., :d_rope], pos, base), x[..., d_rope:]], axis=-1)
+
+
+def decode_attention_decoupled(q, k_self, v_self, c_k, c_v, W_up_k_t, W_up_v_t, mu_k_t, mu_v_t,
+                               positions, q_pos, base, d_rope, scale=None):
+    """Decode attention with decoupled RoPE, direct form: rebuild K and V from the
+    latents, rotate the first d_rope dims of every key at its position and of the
+    query (and the in-flight key) at q_pos, attend.  Returns out [d]."""
+    q = np.asarray(q, np.float64)
+    d = q.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    K = reconstruct(c_k, W_up_k_t, mu_k_t).reshape(-1, d)
+    V = reconstruct(c_v, W_up_v_t, mu_v_t).reshape(-1, d)
+    qr = rope_partial(q, q_pos, base, d_rope)
+    Kr = rope_partial(K, np.asarray(positions), base, d_rope)
+    ks = rope_partial(k_self, q_pos, base, d_rope)
+    s = np.concatenate([Kr @ qr, [ks @ qr]]) * scale
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    return p[:-1] @ V + p[-1] * np.asarray(v_self, np.float64)
+
+
+def decode_attention_decoupled_absorbed(q, k_self, v_self, c_k, c_v, W_up_k_t, W_up_v_t, mu_k_t,
+                                        mu_v_t, positions, q_pos, base, d_rope, scale=None):
+    """The same result computed the way App. J describes it: the NoPE content score
+    is taken in latent space with the query absorbed into the up-projection,
+        q_nope . (c W_nope^T + mu_nope) = (W_nope^T q_nope) . c + q_nope . mu_nope,
+    only the d_rope rotary dims of each key are rebuilt and rotated, and values
+    are summed in latent space and up-projected once."""
+    q = np.asarray(q, np.float64)
+    d = q.shape[-1]
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    Wk = np.asarray(W_up_k_t, np.float64)
+    mk = np.asarray(mu_k_t, np.float64)
+    c_k = np.asarray(c_k, np.float64).reshape(-1, Wk.shape[1])
+    q_nope = q[d_rope:]
+    a_nope = Wk[d_rope:].T @ q_nope                    # absorbed query, [r_k]
+    s_hist = c_k @ a_nope + q_nope @ mk[d_rope:]
+    if d_rope:
+        K_rope = c_k @ Wk[:d_rope].T + mk[:d_rope]     # explicit rotary branch only
+        q_rope = rope(q[:d_rope], q_pos, base)
+        s_hist = s_hist + rope(K_rope, np.asarray(positions), base) @ q_rope
+    ks = np.asarray(k_self, np.float64)
+    s_self = float(rope_partial(ks, q_pos, base, d_rope) @ rope_partial(q, q_pos, base, d_rope))
+    s = np.concatenate([s_hist, [s_self]]) * scale
+    p = np.exp(s - s.max())
+    p /= p.sum()
+    Wv = np.asarray(W_up_v_t, np.float64)
+    c_v = np.asarray(c_v, np.float64).reshape(-1, Wv.shape[1])
+    o_lat = p[:-1] @ c_v
+    return (o_lat @ Wv.T + p[:-1].sum() * np.asarray(mu_v_t, np.float64)
+            + p[-1] * np.asarray(v_self, np.float64))
+
+
+def decode_attn_cache_decoupled(cfg: Cfg, codec: Codec, t: int, q, k_self, v_self, c_k, c_v,
+                                positions, q_pos, ctx_len, d_rope, pairs=None, scale=None):
+    """``decode_attention_decoupled`` for a batch in the library's layout (see
+    ``decode_attn_cache``).  Returns out [B, H, d] (NaN outside ``pairs``)."""
+    q = np.asarray(q, np.float64)
+    B, H, d = q.shape
+    out = np.full((B, H, d), np.nan)
+    if pairs is None:
+        pairs = [(b, h) for b in range(B) for h in range(H)]
+    for b, h in pairs:
+        n = int(ctx_len[b])
+        if cfg.mode == MODE_PER_HEAD:
+            ck, cv = np.asarray(c_k[b, :n, h]), np.asarray(c_v[b, :n, h])
+        else:
+            ck, cv = np.asarray(c_k[b, :n]), np.asarray(c_v[b, :n])
+        out[b, h] = decode_attention_decoupled(
+            q[b, h], k_self[b, h], v_self[b, h], ck, cv, w_up_t(cfg, codec.W_up_k, t, h),
+            w_up_t(cfg, codec.W_up_v, t, h), mu_t(cfg, codec.mu_k, t, h),
+            mu_t(cfg, codec.mu_v, t, h), np.asarray(positions[b, :n]), int(q_pos[b]),
+            cfg.rope_base, d_rope, scale)
+    return out
