@@ -68,7 +68,8 @@ extern "C" {
 /*
  * Codec geometry of one shared layer.
  * Supported: 1 <= T <= 64; 1 <= H <= 128; d_head in {32, 64, 96, 128};
- * r_k, r_v multiples of 8 in [8, 256]; rope_base > 1; sm_scale >= 0.
+ * r_k, r_v multiples of 8 in [8, 256]; rope_base > 1; sm_scale >= 0;
+ * d_rope in {0, 32, 64, d_head} (see the field).
  */
 typedef struct lla_cfg {
   int32_t T;        /* loops */
@@ -79,6 +80,13 @@ typedef struct lla_cfg {
   int32_t mode;     /* LLA_MODE_PER_HEAD or LLA_MODE_2D */
   float rope_base;  /* RoPE base, e.g. 10000 */
   float sm_scale;   /* softmax scale; 0 selects 1/sqrt(d_head) */
+  int32_t d_rope;   /* 0: RoPE over the whole head (the method's default).  Otherwise the
+                       decoupled RoPE of the close reading, Appendix J: only the first
+                       d_rope dims of q and k rotate, as a rotary vector of their own width
+                       (pairs (i, i + d_rope/2), angle pos * rope_base^(-2 i / d_rope)),
+                       and the other dims form a NoPE content path that decode absorbs into
+                       the query.  Supported: 32 or 64, below d_head, per-head mode, decode
+                       on the tensor-core path; d_rope == d_head is the default RoPE. */
 } lla_cfg;
 
 /* Last error message of the calling thread ("" if none). Never NULL. */

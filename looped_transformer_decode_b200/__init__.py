@@ -83,7 +83,8 @@ def codec_pack(cfg: Cfg, W_down_k, W_down_v, W_up_k, W_up_v, mu_k, mu_v, out=Non
 def rope_table(cfg: Cfg, max_pos: int, device="cuda", out=None):
     c = cfg.c()
     if out is None:
-        out = torch.empty((max_pos, cfg.d_head // 2, 2), dtype=torch.float32, device=device)
+        rd = cfg.d_rope or cfg.d_head                 # rotary dims
+        out = torch.empty((max_pos, rd // 2, 2), dtype=torch.float32, device=device)
     check(lib.lla_rope_table(ctypes.byref(c), max_pos, _ptr(out, torch.float32, "table"),
                              out.numel() * 4, _stream()))
     return out

@@ -32,7 +32,8 @@ class LLAError(RuntimeError):
 class CCfg(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("d_head", ctypes.c_int32),
                 ("r_k", ctypes.c_int32), ("r_v", ctypes.c_int32), ("mode", ctypes.c_int32),
-                ("rope_base", ctypes.c_float), ("sm_scale", ctypes.c_float)]
+                ("rope_base", ctypes.c_float), ("sm_scale", ctypes.c_float),
+                ("d_rope", ctypes.c_int32)]
 
 
 @dataclass(frozen=True)
@@ -45,10 +46,11 @@ class Cfg:
     mode: int = MODE_PER_HEAD
     rope_base: float = 10000.0
     sm_scale: float = 0.0
+    d_rope: int = 0          # decoupled RoPE: rotary dims (0 = the whole head)
 
     def c(self) -> CCfg:
         return CCfg(self.T, self.H, self.d_head, self.r_k, self.r_v, self.mode, self.rope_base,
-                    self.sm_scale)
+                    self.sm_scale, self.d_rope)
 
 
 if not os.path.exists(LIB_PATH):

@@ -46,6 +46,10 @@ int check_cfg(const lla_cfg* c) {
     return fail(LLA_ERR_INVALID, "rope_base=%g must be a finite value > 1", (double)c->rope_base);
   if (!(c->sm_scale >= 0.0f) || !std::isfinite(c->sm_scale))
     return fail(LLA_ERR_INVALID, "sm_scale=%g must be finite and >= 0", (double)c->sm_scale);
+  if (c->d_rope != 0 && c->d_rope != c->d_head && c->d_rope != 32 && c->d_rope != 64)
+    return fail(LLA_ERR_UNSUPPORTED, "d_rope=%d not in {0, 32, 64, d_head}", c->d_rope);
+  if (c->d_rope > c->d_head)
+    return fail(LLA_ERR_INVALID, "d_rope=%d above d_head=%d", c->d_rope, c->d_head);
   return LLA_OK;
 }
 
@@ -207,7 +211,7 @@ int lla_codec_pack(const lla_cfg* cfg, const float* W_down_k, const float* W_dow
 size_t lla_rope_table_bytes(const lla_cfg* cfg, int32_t max_pos) {
   if (check_cfg(cfg) || max_pos < 0) return 0;
   ok();
-  return (size_t)max_pos * (cfg->d_head / 2) * sizeof(float2);
+  return (size_t)max_pos * (rotary_dims(*cfg) / 2) * sizeof(float2);
 }
 
 int lla_rope_table(const lla_cfg* cfg, int32_t max_pos, void* table, size_t table_bytes,
@@ -302,6 +306,10 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
     }
   }
   SplitPlan plan = split_plan(*cfg, B, n_cap);
+  if (has_nope(*cfg) && n_cap > 0 && !plan.tensor_cores)
+    return fail(LLA_ERR_UNSUPPORTED,
+                "decoupled RoPE (d_rope=%d) runs on the per-head tensor-core path only",
+                cfg->d_rope);
   const size_t ops_at = kWsHeader + align_up(partials_bytes(*cfg, B, plan.splits), 256);
   const size_t counters_at = ops_at + align_up(plan.ops_bytes, 256);
   size_t need = counters_at + (plan.tensor_cores ? align_up(((size_t)B * cfg->H + 1) * 4, 256) : 0);
@@ -315,6 +323,7 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   a.T = cfg->T;
   a.H = cfg->H;
   a.d = cfg->d_head;
+  a.rd = rotary_dims(*cfg);
   a.r_k = cfg->r_k;
   a.r_v = cfg->r_v;
   a.mode = cfg->mode;
@@ -362,6 +371,8 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   cudaError_t ce = cudaErrorNotSupported;
   if (plan.tensor_cores && plan.splits > 0)
     ce = launch_decode_tc(*cfg, a, static_cast<cudaStream_t>(stream));
+  if (ce == cudaErrorNotSupported && has_nope(*cfg) && n_cap > 0)
+    return fail(LLA_ERR_UNSUPPORTED, "decoupled RoPE shape not taken by the tensor-core path");
   if (ce == cudaErrorNotSupported) ce = launch_decode(a, static_cast<cudaStream_t>(stream), &launches);
   if (ce != cudaSuccess) return cuda_fail(ce, "lla_decode_attn launch");
   return ok();
@@ -405,6 +416,7 @@ int lla_full_rebuild(const lla_cfg* cfg, const void* packed, const void* rope_ta
                      int32_t* status, void* stream) {
   int e = check_cfg(cfg);
   if (e) return e;
+  if (has_nope(*cfg)) return fail(LLA_ERR_UNSUPPORTED, "the full-memory path rotates whole heads");
   if (t < 0 || t >= cfg->T) return fail(LLA_ERR_INVALID, "t=%d outside [0, T=%d)", t, cfg->T);
   if (B < 0 || n_cap < 0 || n_rows < 0)
     return fail(LLA_ERR_INVALID, "B, n_cap and n_rows must be >= 0");
@@ -475,6 +487,7 @@ int lla_full_decode_attn(const lla_cfg* cfg, const void* rope_table, int32_t rop
                          size_t ws_bytes, void* stream) {
   int e = check_cfg(cfg);
   if (e) return e;
+  if (has_nope(*cfg)) return fail(LLA_ERR_UNSUPPORTED, "the full-memory path rotates whole heads");
   if (B < 0 || n_cap < 0) return fail(LLA_ERR_INVALID, "B and n_cap must be >= 0");
   if (rope_max_pos < 1) return fail(LLA_ERR_INVALID, "rope_max_pos must be >= 1");
   if ((long long)B * cfg->H * (long long)n_cap > (long long)INT32_MAX)

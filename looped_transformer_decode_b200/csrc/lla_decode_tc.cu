@@ -301,12 +301,17 @@ __device__ __forceinline__ int checked_pos(const TcParams& p, int pos) {
 // no-swizzle K-major shared-memory layout, and the bias tile image (K column 0 =
 // bf16 hi part of M~, column 1 = lo part).  One CTA of 128 threads per (h, b).
 template <int D>
+// D: rotated dims (the head, or the decoupled rotary branch).  With decoupled RoPE
+// (d_full > D) the images get 16 more rows: row D is the NoPE content path with the
+// query absorbed, kappa sum_{e >= D} q_e W_up,k[e][k] (bias kappa q_nope . mu_nope),
+// and rows D + 1 .. D + 15 are zero.
 __global__ void __launch_bounds__(128) decode_prep_kernel(
     const float* __restrict__ q, const int32_t* __restrict__ q_pos, const float2* __restrict__ rope,
     int rope_max_pos, const float* __restrict__ wupk_t, const float* __restrict__ muk_t, float kappa,
     int H, int r_k, int K_pad, unsigned char* __restrict__ ops_b,
-    unsigned char* __restrict__ ops_bias, int32_t* status, uint32_t* counters) {
+    unsigned char* __restrict__ ops_bias, int32_t* status, uint32_t* counters, int d_full) {
   constexpr int HALF = D / 2;
+  const int NS = d_full > D ? D + 16 : D;      // rows of the images
   __shared__ float2 qc[HALF];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   // the CTA counter of the fused-combine kernels starts every call at zero (this
@@ -318,50 +323,71 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
     if (tid == 0 && h == 0 && blockIdx.z == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
     qp = 0;
   }
-  const float* qh = q + ((size_t)b * H + h) * D;
+  const float* qh = q + ((size_t)b * H + h) * d_full;
   for (int i = tid; i < HALF; i += blockDim.x) {
     const float2 e = rope[(size_t)qp * HALF + i];
     const float x0 = qh[i], x1 = qh[i + HALF];
     qc[i] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
   }
   __syncthreads();
-  const float* W = wupk_t + (size_t)h * D * r_k;  // [d][r_k]
-  unsigned char* img = ops_b + ((size_t)b * H + h) * (size_t)D * K_pad * 2;
+  const float* W = wupk_t + (size_t)h * d_full * r_k;  // [d][r_k]
+  unsigned char* img = ops_b + ((size_t)b * H + h) * (size_t)NS * K_pad * 2;
   // One 16-byte chunk (8 consecutive K values of one row n) per iteration.
-  const int chunks = D * K_pad / 8;
+  const int chunks = NS * K_pad / 8;
   for (int c = blockIdx.z * blockDim.x + tid; c < chunks; c += gridDim.z * blockDim.x) {
     const int n = (c / K_pad) * 8 + (c & 7);
     const int k0 = ((c >> 3) % (K_pad / 8)) * 8;
-    const int i = n >> 1;
-    const float2 z = qc[i];
     __align__(16) __nv_bfloat16 v[8];
+    if (n < D) {
+      const int i = n >> 1;
+      const float2 z = qc[i];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int k = k0 + e;
-      float val = 0.f;
-      if (k < r_k) {
-        const float wr = W[(size_t)i * r_k + k], wi = W[(size_t)(i + HALF) * r_k + k];
-        val = (n & 1) ? kappa * (z.x * wi - z.y * wr) : kappa * (z.x * wr + z.y * wi);
+      for (int e = 0; e < 8; ++e) {
+        const int k = k0 + e;
+        float val = 0.f;
+        if (k < r_k) {
+          const float wr = W[(size_t)i * r_k + k], wi = W[(size_t)(i + HALF) * r_k + k];
+          val = (n & 1) ? kappa * (z.x * wi - z.y * wr) : kappa * (z.x * wr + z.y * wi);
+        }
+        v[e] = __float2bfloat16_rn(val);
       }
-      v[e] = __float2bfloat16_rn(val);
+    } else {
+      // NoPE content path: the query absorbed into the unrotated dims' up-projection
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int k = k0 + e;
+        float val = 0.f;
+        if (n == D && k < r_k) {
+          for (int dd = D; dd < d_full; ++dd) val = fmaf(qh[dd], W[(size_t)dd * r_k + k], val);
+          val *= kappa;
+        }
+        v[e] = __float2bfloat16_rn(val);
+      }
     }
     *reinterpret_cast<uint4*>(img + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
   }
   // Bias tile image [D x 16]: chunk c covers row n = (c / 2 / 8) * 8 + c % 8 ... laid out as
   // core matrices (n / 8, k / 8) at (n / 8) * 256 + (k / 8) * 128 + (n % 8) * 16.
-  unsigned char* bimg = ops_bias + ((size_t)b * H + h) * (size_t)D * 32;
-  const float* mu = muk_t + (size_t)h * D;
-  for (int c = blockIdx.z * blockDim.x + tid; c < D * 2; c += gridDim.z * blockDim.x) {
+  unsigned char* bimg = ops_bias + ((size_t)b * H + h) * (size_t)NS * 32;
+  const float* mu = muk_t + (size_t)h * d_full;
+  for (int c = blockIdx.z * blockDim.x + tid; c < NS * 2; c += gridDim.z * blockDim.x) {
     const int n = (c >> 4) * 8 + (c & 7);
     const int kc = (c >> 3) & 1;
     __align__(16) __nv_bfloat16 v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = __float2bfloat16_rn(0.f);
-    if (kc == 0) {
-      const int i = n >> 1;
-      const float2 z = qc[i];
-      const float mr = mu[i], mi = mu[i + HALF];
-      const float val = (n & 1) ? kappa * (z.x * mi - z.y * mr) : kappa * (z.x * mr + z.y * mi);
+    if (kc == 0 && n <= D && (n < D || d_full > D)) {
+      float val;
+      if (n < D) {
+        const int i = n >> 1;
+        const float2 z = qc[i];
+        const float mr = mu[i], mi = mu[i + HALF];
+        val = (n & 1) ? kappa * (z.x * mi - z.y * mr) : kappa * (z.x * mr + z.y * mi);
+      } else {
+        val = 0.f;
+        for (int dd = D; dd < d_full; ++dd) val = fmaf(qh[dd], mu[dd], val);
+        val *= kappa;
+      }
       v[0] = __float2bfloat16_rn(val);
       v[1] = __float2bfloat16_rn(val - __bfloat162float(v[0]));
     }
@@ -444,10 +470,14 @@ __device__ void combine_head(const TcParams& p, int b, int h, unsigned char* scr
   named_barrier(bar, 128);   // scratch is reused by the next head
 }
 
-template <int D, int G, bool FUSE>
+// D: rotated dims per head.  NOPE (decoupled RoPE): each head's score operand has
+// 16 more columns, the first of which is the NoPE content score (read by
+// warpgroup 0 and added to the rotary branch's score).
+template <int D, int G, bool FUSE, bool NOPE>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
+  constexpr int NS = D + (NOPE ? 16 : 0);   // score columns per head
   constexpr int HALF = D / 2;
   constexpr int WG_PAIRS = HALF / kEpiWG;   // RoPE pairs per epilogue warpgroup
   constexpr int WG_COLS = 2 * WG_PAIRS;     // TMEM columns per warpgroup (Re, Im interleaved)
@@ -608,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ score MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, D);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, NS);
       const uint32_t sbo_a = 16u * p.box_k;
       const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 0, 0);   // rows alias
       uint32_t it = 0, jn = 0;
@@ -636,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t st_addr = smem_addr(sm + p.st_off + stage * p.st_bytes);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const uint32_t d_tmem = tmem_base + acc * p.acc_cols + g * D;
+            const uint32_t d_tmem = tmem_base + acc * p.acc_cols + g * NS;
             const uint32_t b_addr = b_base + g * ops_head_bytes;
             for (int kk = 0; kk < p.K_pad / 16; ++kk) {
               const int kb = (kk * 16) / p.box_k, kin = (kk * 16) % p.box_k;
@@ -764,11 +794,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         float part[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const uint32_t col = tmem_base + lane_addr + acc * p.acc_cols + g * D + wgi * WG_COLS;
+          const uint32_t head_col = tmem_base + lane_addr + acc * p.acc_cols + g * NS;
+          const uint32_t col = head_col + wgi * WG_COLS;
           float u[WG_COLS];
 #pragma unroll
           for (int c = 0; c < WG_COLS / 16; ++c) tmem_ld16(col + c * 16, u + c * 16);
           if constexpr (WG_COLS % 16 != 0) tmem_ld8(col + (WG_COLS / 16) * 16, u + (WG_COLS / 16) * 16);
+          float un[8];
+          un[0] = 0.f;
+          if constexpr (NOPE) {
+            if (wgi == 0) tmem_ld8(head_col + D, un);   // the NoPE content column (+ 7 zeros)
+          }
           tmem_wait_ld();
           float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -776,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             a0 = ffma2(make_float2(u[2 * q], u[2 * q + 1]), ef[q], a0);
             if (q + 1 < WG_PAIRS) a1 = ffma2(make_float2(u[2 * q + 2], u[2 * q + 3]), ef[q + 1], a1);
           }
-          part[g] = (a0.x + a0.y) + (a1.x + a1.y);
+          part[g] = (a0.x + a0.y) + (a1.x + a1.y) + un[0];
         }
         tc_fence_before();
         __syncwarp();
@@ -1452,6 +1488,7 @@ struct TcPlan {
   bool ok = false;
   bool shared = false;    // LLA-2D kernel (G heads per item share each latent tile)
   int G = 1, nst = 0, nst_v = 0, nacc = 1, nbuf_b = 2, S = 0, tps = 0;
+  bool nope = false;      // decoupled RoPE: score operands carry a NoPE content column
   size_t ops_bytes = 0;   // workspace for the per-(b, h) operand images
 };
 
@@ -1568,9 +1605,13 @@ uint32_t tc2d_layout(TcParams& p, int D, int HP, int nst, int nst_v, int nbuf_b)
 
 TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   TcPlan pl;
-  const int D = c.d_head;
   if (n_cap <= 0 || B <= 0) return pl;
-  if (D != 32 && D != 64 && D != 96 && D != 128) return pl;
+  if (c.d_head != 32 && c.d_head != 64 && c.d_head != 96 && c.d_head != 128) return pl;
+  // score columns per head: the rotated dims, plus 16 (the NoPE content column and
+  // zero padding) with decoupled RoPE, which only the per-head kernel takes
+  const bool nope = has_nope(c);
+  if (nope && c.mode == LLA_MODE_2D) return pl;
+  const int D = nope ? rotary_dims(c) + 16 : c.d_head;
   const int forced_g = env_int("LLA_TC_G", 0), forced_nst = env_int("LLA_TC_NST", 0);
   const int N_v = (c.r_v + 15) / 16 * 16;
   // Largest head group G whose TMEM columns (score accumulators plus V accumulators)
@@ -1685,6 +1726,7 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   pl.S = (n_tiles + pl.tps - 1) / pl.tps;
   const size_t K_pad = (c.r_k + 15) / 16 * 16;
   pl.ops_bytes = (size_t)B * c.H * ((size_t)D * K_pad * 2 + (size_t)D * 32);
+  pl.nope = nope;
   pl.ok = true;
   return pl;
 }
@@ -1694,11 +1736,14 @@ bool tc_enabled() {
   return !(v && std::strcmp(v, "cuda_core") == 0);
 }
 
-template <int D, int G, bool SHARED>
+template <int D, int G, bool SHARED, bool NOPE>
 cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
                         uint32_t smem, int grid, cudaStream_t s) {
-  auto kern = SHARED ? (p.fuse_combine ? decode_tc2d_kernel<D, G, true> : decode_tc2d_kernel<D, G, false>)
-                     : (p.fuse_combine ? decode_tc_kernel<D, G, true> : decode_tc_kernel<D, G, false>);
+  void (*kern)(CUtensorMap, CUtensorMap, TcParams);
+  if constexpr (SHARED)
+    kern = p.fuse_combine ? decode_tc2d_kernel<D, G, true> : decode_tc2d_kernel<D, G, false>;
+  else
+    kern = p.fuse_combine ? decode_tc_kernel<D, G, true, NOPE> : decode_tc_kernel<D, G, false, NOPE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, SHARED ? kThreads2 : kThreads, smem, s>>>(mk, mv, p);
@@ -1709,26 +1754,39 @@ template <int D>
 cudaError_t launch_tc_d(int G, bool shared, const CUtensorMap& mk, const CUtensorMap& mv,
                         const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
   switch (G * 2 + (shared ? 1 : 0)) {
-    case 2: return launch_tc_t<D, 1, false>(mk, mv, p, smem, grid, s);
-    case 4: return launch_tc_t<D, 2, false>(mk, mv, p, smem, grid, s);
-    case 8: return launch_tc_t<D, 4, false>(mk, mv, p, smem, grid, s);
-    case 3: return launch_tc_t<D, 1, true>(mk, mv, p, smem, grid, s);
-    case 5: return launch_tc_t<D, 2, true>(mk, mv, p, smem, grid, s);
-    case 9: return launch_tc_t<D, 4, true>(mk, mv, p, smem, grid, s);
+    case 2: return launch_tc_t<D, 1, false, false>(mk, mv, p, smem, grid, s);
+    case 4: return launch_tc_t<D, 2, false, false>(mk, mv, p, smem, grid, s);
+    case 8: return launch_tc_t<D, 4, false, false>(mk, mv, p, smem, grid, s);
+    case 3: return launch_tc_t<D, 1, true, false>(mk, mv, p, smem, grid, s);
+    case 5: return launch_tc_t<D, 2, true, false>(mk, mv, p, smem, grid, s);
+    case 9: return launch_tc_t<D, 4, true, false>(mk, mv, p, smem, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Decoupled RoPE (per-head kernel only): D is the rotary branch width.
+template <int D>
+cudaError_t launch_tc_nope(int G, const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
+                           uint32_t smem, int grid, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_tc_t<D, 1, false, true>(mk, mv, p, smem, grid, s);
+    case 2: return launch_tc_t<D, 2, false, true>(mk, mv, p, smem, grid, s);
+    case 4: return launch_tc_t<D, 4, false, true>(mk, mv, p, smem, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_prep(const DecodeArgs& a, const TcParams& p, cudaStream_t s) {
-  const int chunks = a.d * p.K_pad / 8;
+  const int ns = a.rd < a.d ? a.rd + 16 : a.d;      // image rows per head
+  const int chunks = ns * p.K_pad / 8;
   dim3 grid((unsigned)a.H, (unsigned)a.B, (unsigned)((chunks + 127) / 128));
   unsigned char* ob = const_cast<unsigned char*>(p.ops_b);
   unsigned char* obias = const_cast<unsigned char*>(p.ops_bias);
 #define LLA_PREP(DD)                                                                          \
   decode_prep_kernel<DD><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, \
                                               a.muk_t, a.kappa, a.H, a.r_k, p.K_pad, ob, obias, \
-                                              a.status, a.counters)
-  switch (a.d) {
+                                              a.status, a.counters, a.d)
+  switch (a.rd) {
     case 32: LLA_PREP(32); break;
     case 64: LLA_PREP(64); break;
     case 96: LLA_PREP(96); break;
@@ -1775,8 +1833,9 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.r_k = a.r_k;
   p.r_v = a.r_v;
   // At least 120 KB so that two CTAs never share an SM (each may hold all of TMEM).
+  const int ns = pl.nope ? a.rd + 16 : a.d;   // score columns per head
   uint32_t smem = pl.shared ? tc2d_layout(p, a.d, pl.G, pl.nst, pl.nst_v, pl.nbuf_b)
-                            : tc_layout(p, a.d, pl.G, pl.nst, pl.nst_v);
+                            : tc_layout(p, ns, pl.G, pl.nst, pl.nst_v);
   if (smem < 120u * 1024u) smem = 120u * 1024u;
   p.B = a.B;
   p.n_cap = a.n_cap;
@@ -1786,15 +1845,15 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.n_items = a.B * p.HG * pl.S;
   p.rope_max_pos = a.rope_max_pos;
   p.nacc = pl.nacc;
-  p.acc_cols = pl.shared ? a.d : pl.G * a.d;
+  p.acc_cols = pl.shared ? a.d : pl.G * ns;
   p.v_col0 = p.nacc * p.acc_cols;
   const int v_cols = pl.shared ? p.m_v * p.n_p : pl.G * p.N_v;
   int cols = 32;
   while (cols < p.v_col0 + v_cols) cols <<= 1;
   p.tmem_cols = cols;
   p.rope = a.rope;
-  for (int i = 0; i < a.d / 2; ++i) {
-    const double theta = std::pow((double)a.rope_base, -2.0 * i / (double)a.d);
+  for (int i = 0; i < a.rd / 2; ++i) {
+    const double theta = std::pow((double)a.rope_base, -2.0 * i / (double)a.rd);
     const double turns = theta / (2.0 * 3.14159265358979323846);
     const uint64_t fx = static_cast<uint64_t>(std::ldexp(turns - std::floor(turns), 64));
     p.phi_lo[i] = static_cast<uint32_t>(fx);
@@ -1844,12 +1903,20 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   if (pe != cudaSuccess) return pe;
   const int grid = p.n_items < sms ? p.n_items : sms;
   cudaError_t e;
-  switch (a.d) {
-    case 32: e = launch_tc_d<32>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
-    case 64: e = launch_tc_d<64>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
-    case 96: e = launch_tc_d<96>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
-    case 128: e = launch_tc_d<128>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
-    default: return cudaErrorNotSupported;
+  if (pl.nope) {
+    switch (a.rd) {
+      case 32: e = launch_tc_nope<32>(pl.G, mk, mv, p, smem, grid, s); break;
+      case 64: e = launch_tc_nope<64>(pl.G, mk, mv, p, smem, grid, s); break;
+      default: return cudaErrorNotSupported;
+    }
+  } else {
+    switch (a.d) {
+      case 32: e = launch_tc_d<32>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+      case 64: e = launch_tc_d<64>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+      case 96: e = launch_tc_d<96>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+      case 128: e = launch_tc_d<128>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+      default: return cudaErrorNotSupported;
+    }
   }
   if (e == cudaSuccess && !p.fuse_combine) e = launch_combine(a, s);
   return e;

@@ -44,6 +44,10 @@ inline int encode_kc(const lla_cfg& c) {
   return unit % 64 == 0 ? 64 : 32;
 }
 inline int pad16(int r) { return (r + 15) / 16 * 16; }
+// Dims of q and k that RoPE rotates: the whole head, or the decoupled branch.
+inline int rotary_dims(const lla_cfg& c) { return c.d_rope ? c.d_rope : c.d_head; }
+// Decoupled RoPE with a NoPE content path (d_rope below d_head).
+inline bool has_nope(const lla_cfg& c) { return c.d_rope != 0 && c.d_rope < c.d_head; }
 
 // Decode split plan shared by the workspace sizing and the launcher.
 struct SplitPlan {
@@ -79,6 +83,7 @@ cudaError_t launch_evict_append(int B, int n_cap, int sink, int window, const in
 
 struct DecodeArgs {
   int T, H, d, r_k, r_v, mode;
+  int rd;                // rotated dims: d, or the decoupled rotary branch's d_rope
   float kappa;           // sm_scale * log2(e): scores are kept in base-2 units
   int t, B, n_cap, rope_max_pos;
   float rope_base;

@@ -459,7 +459,7 @@ size_t decode_partial_smem(const DecodeArgs& a) {
 }  // namespace
 
 cudaError_t launch_rope_table(const lla_cfg& c, int max_pos, float2* table, cudaStream_t s) {
-  const int half = c.d_head / 2;
+  const int half = rotary_dims(c) / 2;
   const long long n = (long long)max_pos * half;
   const int threads = 256;
   const long long blocks = (n + threads - 1) / threads;

@@ -4,11 +4,15 @@ first d_rope dims of each head.
 
 CPU: the oracle pinned to the full-RoPE decode (d_rope = d), to a NoPE attention
 written out by hand (d_rope = 0), to its own absorbed form, and to the
-relative-position property of the rotary branch.
+relative-position property of the rotary branch; host checks of the ABI.
+GPU: the per-head tensor-core decode with d_rope in {32, 64} against the oracle
+(ragged and random-position cases, several splits and one split per head), and
+the refusal of shapes outside that path.
 """
 from __future__ import annotations
 
 import numpy as np
+import pytest
 
 import oracle as O
 import synth
@@ -93,3 +97,123 @@ def test_only_the_leading_dims_rotate_on_their_own_frequency_ladder():
         np.testing.assert_allclose(y[i], a * np.cos(ang) - b * np.sin(ang), rtol=1e-14, atol=1e-14)
         np.testing.assert_allclose(y[i + d_rope // 2], a * np.sin(ang) + b * np.cos(ang),
                                    rtol=1e-14, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- C ABI, host
+
+def test_decoupled_rope_host_checks():
+    import ctypes
+
+    import looped_transformer_decode_b200 as lla
+
+    def cfg_rc(**kw):
+        c = lla.Cfg(4, 16, 128, 96, 160, **kw)
+        return lla.lib.lla_codec_packed_bytes(ctypes.byref(c.c()))
+    assert cfg_rc(d_rope=64) > 0 and cfg_rc(d_rope=32) > 0 and cfg_rc(d_rope=128) > 0
+    assert cfg_rc(d_rope=48) == 0                       # unsupported width
+    c = lla.Cfg(4, 4, 32, 16, 16, d_rope=64)            # wider than the head
+    assert lla.lib.lla_codec_packed_bytes(ctypes.byref(c.c())) == 0
+    # the RoPE table holds the rotary branch's pairs only
+    for dr, half in ((0, 64), (64, 32), (32, 16), (128, 64)):
+        c = lla.Cfg(4, 16, 128, 96, 160, d_rope=dr)
+        assert lla.lib.lla_rope_table_bytes(ctypes.byref(c.c()), 10) == 10 * half * 8
+    # the full-memory path rotates whole heads
+    p = ctypes.c_void_p(0x1000)
+    c = lla.Cfg(4, 16, 128, 96, 160, d_rope=64).c()
+    assert lla.lib.lla_full_decode_attn(ctypes.byref(c), p, 1, 2, 16, p, p, p, p, p, p, p, p, p,
+                                        1 << 20, None) == lla.ERR_UNSUPPORTED
+
+
+# ----------------------------------------------------------------------------- GPU
+
+def _dev_cfg(cfg, d_rope):
+    import looped_transformer_decode_b200 as lla
+    return lla.Cfg(cfg.T, cfg.H, cfg.d, cfg.r_k, cfg.r_v, cfg.mode, cfg.rope_base, d_rope=d_rope)
+
+
+def _run_decoupled(case, d_rope, t, ws=None):
+    import torch
+
+    import looped_transformer_decode_b200 as lla
+    from gpu_util import bf16_tensor, f32_tensor, i32_tensor, pack
+    lc = _dev_cfg(case.cfg, d_rope)
+    mp = int(max(case.positions.max(initial=0), case.q_pos.max())) + 1
+    rope = lla.rope_table(lc, mp)
+    if ws is None:
+        ws = lla.decode_workspace(lc, case.B, case.n_cap)
+    out = lla.decode_attn(lc, pack(case), rope, t, i32_tensor(case.ctx_len), f32_tensor(case.q),
+                          f32_tensor(case.k_self[t]), f32_tensor(case.v_self[t]),
+                          i32_tensor(case.positions), i32_tensor(case.q_pos),
+                          bf16_tensor(case.c_k), bf16_tensor(case.c_v), ws=ws)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy(), ws
+
+
+DECOUPLED_CASES = [
+    (O.Cfg(4, 2, 128, 96, 160), 64, [300, 129, 1], "random"),
+    (O.Cfg(4, 4, 128, 16, 32), 32, [200, 64], "arange"),
+    (O.Cfg(2, 2, 96, 32, 48), 64, [130, 7], "random"),
+    (O.Cfg(2, 4, 64, 24, 40), 32, [100], "random"),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("spec", DECOUPLED_CASES, ids=lambda s: f"d{s[0].d}r{s[1]}n{max(s[2])}")
+def test_decoupled_decode_matches_oracle(spec):
+    from cases import ATTN_TOL, decode_case, rel_err
+    cfg, d_rope, ctx, pos_kind = spec
+    ctx = np.asarray(ctx)
+    case = decode_case(cfg, len(ctx), int(ctx.max()), seed=900 + d_rope + cfg.d, ctx_len=ctx,
+                       positions=pos_kind, codec="random")
+    for t in (0, cfg.T - 1):
+        got, ws = _run_decoupled(case, d_rope, t)
+        want = O.decode_attn_cache_decoupled(cfg, case.codec, t, case.q, case.k_self[t],
+                                             case.v_self[t], case.c_k, case.c_v, case.positions,
+                                             case.q_pos, case.ctx_len, d_rope)
+        assert np.isfinite(got).all()
+        assert rel_err(got, want).max() <= ATTN_TOL, (t, rel_err(got, want).max())
+        # and the kernel follows the decoupled scores, not full RoPE (the two outputs
+        # differ by ~1e-3 here; the kernel sits ten times closer to the decoupled one)
+        full = O.decode_attn_cache(cfg, case.codec, t, case.q, case.k_self[t], case.v_self[t],
+                                   case.c_k, case.c_v, case.positions, case.q_pos, case.ctx_len)
+        assert 10 * rel_err(got, want).max() < rel_err(got, full).max()
+        import looped_transformer_decode_b200 as lla
+        assert lla.decode_status(ws) == 0
+
+
+@pytest.mark.gpu
+def test_decoupled_one_split_per_head_plan():
+    """Enough heads for one split each: the combine runs inside the partial kernel."""
+    from cases import ATTN_TOL, decode_case, rel_err
+
+    import looped_transformer_decode_b200 as lla
+    cfg = O.Cfg(4, 16, 128, 96, 160)
+    ctx = np.array([260, 255, 129, 1, 0, 200, 256, 77] * 2)
+    lc = _dev_cfg(cfg, 64)
+    assert lla.decode_launches(lc, len(ctx), int(ctx.max())) == 2
+    case = decode_case(cfg, len(ctx), int(ctx.max()), seed=950, ctx_len=ctx, positions="random",
+                       codec="random")
+    got, _ = _run_decoupled(case, 64, 1)
+    want = O.decode_attn_cache_decoupled(cfg, case.codec, 1, case.q, case.k_self[1],
+                                         case.v_self[1], case.c_k, case.c_v, case.positions,
+                                         case.q_pos, case.ctx_len, 64)
+    assert rel_err(got, want).max() <= ATTN_TOL
+
+
+@pytest.mark.gpu
+def test_decoupled_rope_outside_the_tensor_core_path_is_refused(monkeypatch):
+    import torch
+
+    import looped_transformer_decode_b200 as lla
+    from cases import decode_case
+    cfg = O.Cfg(2, 2, 64, 16, 16)
+    case = decode_case(cfg, 1, 40, seed=960, codec="random")
+    monkeypatch.setenv("LLA_DECODE_PATH", "cuda_core")
+    with pytest.raises(lla.LLAError):
+        _run_decoupled(case, 32, 0)
+    cfg2 = O.Cfg(2, 4, 64, 16, 16, O.MODE_2D)
+    case2 = decode_case(cfg2, 1, 40, seed=961, codec="random")
+    monkeypatch.delenv("LLA_DECODE_PATH")
+    with pytest.raises(lla.LLAError):
+        _run_decoupled(case2, 32, 0)
+    torch.cuda.synchronize()
