@@ -40,6 +40,8 @@ NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 277.77e6,
                "deeploop_32x_T32_H8_d96_r64_128_B16_n32768": 55.24e9}
 # The same for the full-memory fast path (dominant kernel: full_decode_kernel).
 NCU_TRAFFIC_FULL = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 272.19e6}
+# The same for decoupled RoPE (--d-rope), keyed by (workload, d_rope).
+NCU_TRAFFIC_DECOUPLED = {("perhead_4x_T4_H16_d128_r96_160_B8_n4096", 64): 276.32e6}
 
 
 def parse():
@@ -58,6 +60,9 @@ def parse():
                    help="latent: decode over the latent cache (rebuild on read); full: the "
                         "full-memory fast path (K/V rebuilt once per token into a full bf16 "
                         "cache per loop, ordinary attention)")
+    p.add_argument("--d-rope", type=int, default=0,
+                   help="decoupled RoPE: rotate only the first D_ROPE dims of each head and "
+                        "absorb the rest into a NoPE content path (32 or 64; 0 = whole head)")
     p.add_argument("--evict", default="",
                    help="SINK,WINDOW: decode over a sink + window retention budget of the "
                         "history (eviction composed with the latent cache)")
@@ -177,11 +182,11 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def build_state(w, device):
+def build_state(w, device, d_rope=0):
     import torch
     import looped_transformer_decode_b200 as lla
 
-    cfg = lla.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
+    cfg = lla.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode, d_rope=d_rope)
     append = w.encode_tokens <= w.B               # decode-time append: one new row per sequence
     n_cap = w.n + 1 if append else w.n
     layers = []
@@ -324,7 +329,7 @@ def barrier_sync(dist_on):
     torch.cuda.synchronize()
 
 
-def cpu_baseline_sample(w, seconds: float, loops=None):
+def cpu_baseline_sample(w, seconds: float, loops=None, d_rope=0):
     """Time the float64 oracle on (b, h) pairs of the workload at full context."""
     import torch
     import oracle as O
@@ -347,9 +352,14 @@ def cpu_baseline_sample(w, seconds: float, loops=None):
     while True:
         h = pairs % w.H
         t = loops[pairs % len(loops)]
-        O.decode_attn_cache(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"], arr["c_k"],
-                            arr["c_v"], arr["positions"], arr["q_pos"], arr["ctx_len"],
-                            pairs=[(0, h)])
+        if d_rope:
+            O.decode_attn_cache_decoupled(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"],
+                                          arr["c_k"], arr["c_v"], arr["positions"], arr["q_pos"],
+                                          arr["ctx_len"], d_rope, pairs=[(0, h)])
+        else:
+            O.decode_attn_cache(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"], arr["c_k"],
+                                arr["c_v"], arr["positions"], arr["q_pos"], arr["ctx_len"],
+                                pairs=[(0, h)])
         pairs += 1
         el = time.perf_counter() - t0
         if el >= seconds and pairs >= 2:
@@ -379,7 +389,7 @@ def run_gpu(args):
     w = synth.WORKLOADS[args.workload]
     if args.encode_tokens:
         w = dataclasses.replace(w, encode_tokens=args.encode_tokens)
-    st = build_state(w, device)
+    st = build_state(w, device, args.d_rope)
     n_ctx = w.n
     evict = None
     if args.evict:
@@ -486,13 +496,14 @@ def run_gpu(args):
                    "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
                    "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
                    "evict": list(evict) if evict else None, "attended_context": n_ctx,
-                   "path": args.path, "l2": l2_note},
+                   "path": args.path, "d_rope": args.d_rope or None, "l2": l2_note},
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
         "roofline": {"bound": "hbm", "kernel": kname,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": (traffic_table.get(w.name)
+                     "traffic": ((NCU_TRAFFIC_DECOUPLED.get((w.name, args.d_rope))
+                                  if args.d_rope else traffic_table.get(w.name))
                                  if not (args.encode_tokens or args.evict) else None),
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "call_us": round(unit_ms * 1e3, 2),
@@ -510,7 +521,8 @@ def run_gpu(args):
         line["e2e_note"] = "end-to-end line measured on the latent path (the default)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = (cpu_baseline_full(w, args.cpu_seconds) if full
-                                else cpu_baseline_sample(w, args.cpu_seconds))
+                                else cpu_baseline_sample(w, args.cpu_seconds,
+                                                         d_rope=args.d_rope))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:

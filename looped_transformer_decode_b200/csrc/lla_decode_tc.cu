@@ -332,66 +332,100 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
   __syncthreads();
   const float* W = wupk_t + (size_t)h * d_full * r_k;  // [d][r_k]
   unsigned char* img = ops_b + ((size_t)b * H + h) * (size_t)NS * K_pad * 2;
-  // One 16-byte chunk (8 consecutive K values of one row n) per iteration.
-  const int chunks = NS * K_pad / 8;
+  // One 16-byte chunk (8 consecutive K values of one row n) per iteration; rows < D
+  // here, the 16 NoPE rows (decoupled RoPE) below.
+  const int chunks = D * K_pad / 8;
   for (int c = blockIdx.z * blockDim.x + tid; c < chunks; c += gridDim.z * blockDim.x) {
     const int n = (c / K_pad) * 8 + (c & 7);
     const int k0 = ((c >> 3) % (K_pad / 8)) * 8;
     __align__(16) __nv_bfloat16 v[8];
-    if (n < D) {
-      const int i = n >> 1;
-      const float2 z = qc[i];
+    const int i = n >> 1;
+    const float2 z = qc[i];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int k = k0 + e;
-        float val = 0.f;
-        if (k < r_k) {
-          const float wr = W[(size_t)i * r_k + k], wi = W[(size_t)(i + HALF) * r_k + k];
-          val = (n & 1) ? kappa * (z.x * wi - z.y * wr) : kappa * (z.x * wr + z.y * wi);
-        }
-        v[e] = __float2bfloat16_rn(val);
+    for (int e = 0; e < 8; ++e) {
+      const int k = k0 + e;
+      float val = 0.f;
+      if (k < r_k) {
+        const float wr = W[(size_t)i * r_k + k], wi = W[(size_t)(i + HALF) * r_k + k];
+        val = (n & 1) ? kappa * (z.x * wi - z.y * wr) : kappa * (z.x * wr + z.y * wi);
       }
-    } else {
-      // NoPE content path: the query absorbed into the unrotated dims' up-projection
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int k = k0 + e;
-        float val = 0.f;
-        if (n == D && k < r_k) {
-          for (int dd = D; dd < d_full; ++dd) val = fmaf(qh[dd], W[(size_t)dd * r_k + k], val);
-          val *= kappa;
-        }
-        v[e] = __float2bfloat16_rn(val);
-      }
+      v[e] = __float2bfloat16_rn(val);
     }
     *reinterpret_cast<uint4*>(img + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
+  }
+  __shared__ float a_part[4][256];
+  __shared__ float q_nope[128];
+  __shared__ float mu_nope;
+  if (d_full > D && blockIdx.z == 0) {
+    // NoPE content path: the query absorbed into the unrotated dims' up-projection,
+    // a[k] = kappa sum_{dd >= D} q_dd W[dd][k], and its bias kappa q_nope . mu_nope.
+    // Warp w sums a quarter of the dims for every k (lanes over k: coalesced W rows).
+    const int nd = d_full - D, w = tid >> 5, lane = tid & 31;
+    for (int dd = tid; dd < nd; dd += blockDim.x) q_nope[dd] = qh[D + dd];
+    __syncthreads();
+    const int per = (nd + 3) / 4, d0 = w * per, d1 = min(nd, d0 + per);
+    for (int k = lane; k < r_k; k += 32) {
+      float acc = 0.f;
+#pragma unroll 8
+      for (int dd = d0; dd < d1; ++dd) acc = fmaf(q_nope[dd], W[(size_t)(D + dd) * r_k + k], acc);
+      a_part[w][k] = acc;
+    }
+    if (tid < 32) {
+      float acc = 0.f;
+      for (int dd = tid; dd < nd; dd += 32) acc = fmaf(q_nope[dd], muk_t[(size_t)h * d_full + D + dd], acc);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (tid == 0) mu_nope = kappa * acc;
+    }
+    __syncthreads();
+    // rows D .. D + 15: two 8-row groups of K_pad / 8 chunks each; only row D is nonzero
+    for (int c2 = tid; c2 < 2 * K_pad; c2 += blockDim.x) {
+      const int c = (D / 8) * K_pad + c2;
+      const int n = (c / K_pad) * 8 + (c & 7);
+      const int k0 = ((c >> 3) % (K_pad / 8)) * 8;
+      __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        v[e] = __float2bfloat16_rn(n == D && k0 + e < r_k
+                                       ? kappa * ((a_part[0][k0 + e] + a_part[1][k0 + e]) +
+                                                  (a_part[2][k0 + e] + a_part[3][k0 + e]))
+                                       : 0.f);
+      *reinterpret_cast<uint4*>(img + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
+    }
   }
   // Bias tile image [D x 16]: chunk c covers row n = (c / 2 / 8) * 8 + c % 8 ... laid out as
   // core matrices (n / 8, k / 8) at (n / 8) * 256 + (k / 8) * 128 + (n % 8) * 16.
   unsigned char* bimg = ops_bias + ((size_t)b * H + h) * (size_t)NS * 32;
   const float* mu = muk_t + (size_t)h * d_full;
-  for (int c = blockIdx.z * blockDim.x + tid; c < NS * 2; c += gridDim.z * blockDim.x) {
+  for (int c = blockIdx.z * blockDim.x + tid; c < D * 2; c += gridDim.z * blockDim.x) {
     const int n = (c >> 4) * 8 + (c & 7);
     const int kc = (c >> 3) & 1;
     __align__(16) __nv_bfloat16 v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = __float2bfloat16_rn(0.f);
-    if (kc == 0 && n <= D && (n < D || d_full > D)) {
-      float val;
-      if (n < D) {
-        const int i = n >> 1;
-        const float2 z = qc[i];
-        const float mr = mu[i], mi = mu[i + HALF];
-        val = (n & 1) ? kappa * (z.x * mi - z.y * mr) : kappa * (z.x * mr + z.y * mi);
-      } else {
-        val = 0.f;
-        for (int dd = D; dd < d_full; ++dd) val = fmaf(qh[dd], mu[dd], val);
-        val *= kappa;
-      }
+    if (kc == 0) {
+      const int i = n >> 1;
+      const float2 z = qc[i];
+      const float mr = mu[i], mi = mu[i + HALF];
+      const float val = (n & 1) ? kappa * (z.x * mi - z.y * mr) : kappa * (z.x * mr + z.y * mi);
       v[0] = __float2bfloat16_rn(val);
       v[1] = __float2bfloat16_rn(val - __bfloat162float(v[0]));
     }
     *reinterpret_cast<uint4*>(bimg + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
+  }
+  if (d_full > D && blockIdx.z == 0) {
+    // bias rows D .. D + 15: row D carries kappa q_nope . mu_nope as bf16 hi + lo
+    for (int c = 2 * D + tid; c < 2 * NS; c += blockDim.x) {
+      const int n = (c >> 4) * 8 + (c & 7);
+      __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __float2bfloat16_rn(0.f);
+      if (n == D && ((c >> 3) & 1) == 0) {
+        v[0] = __float2bfloat16_rn(mu_nope);
+        v[1] = __float2bfloat16_rn(mu_nope - __bfloat162float(v[0]));
+      }
+      *reinterpret_cast<uint4*>(bimg + (size_t)c * 16) = *reinterpret_cast<const uint4*>(v);
+    }
   }
 }
 
