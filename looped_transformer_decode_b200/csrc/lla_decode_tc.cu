@@ -817,6 +817,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref[g] = -INFINITY;
         l_part[g] = 0.f;
       }
+      // fused finish, set up while the tiles stream: the in-flight scores' partial
+      // dot products q . k_self go to shared memory (per warp of warpgroup 0), and the
+      // heads' W_up,v rows into L2, kept there ahead of the latent stream
+      if constexpr (FUSE) {
+        float* misc = reinterpret_cast<float*>(sm + p.comb_off) + 512;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const size_t bh = (size_t)r.b * p.H + r.hg * G + g;
+          if (wgi == 0) {
+            const float qk = row < p.d ? __ldg(p.q + bh * p.d + row) * __ldg(p.k_self + bh * p.d + row) : 0.f;
+            const float sdot = warp_sum_f(qk);
+            if (lane == 0) misc[8 + g * 4 + sub] = sdot;
+          }
+          const char* wrow = reinterpret_cast<const char*>(p.wupv_t + (size_t)(r.hg * G + g) * p.d * p.r_v);
+          for (int off = et * 128; off < p.d * p.r_v * 4; off += kEpiThreads * 128)
+            asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wrow + off));
+        }
+      }
       for (int k = 0; k < r.ntiles; ++k, ++it) {
         const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
         const int t0 = r.tok0 + k * kTile;
@@ -949,7 +967,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (aborted) break;
       // ---------------------------------------------------------- item partial
-      if (wgi == 0 && r.ntiles > 0) {
+      if constexpr (FUSE) {
+        // One split per group: finish its heads here from on-chip state with both
+        // warpgroups: o = (W_up,v o_lat a + mu_v l a + v_self b) / (l a + b), where
+        // a = 2^(m - M), b = 2^(s_self - M), M = max(m, s_self) (base-2 scores).
+        float* olat = reinterpret_cast<float*>(sm + p.comb_off);   // [r_v]
+        float* yh = olat + 256;                                      // [2][128]
+        float* misc = yh + 256;             // [32]: m per head [0, 4), q . k_self partials [8, 24)
+        if (wgi == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float l = warp_sum_f(l_part[g]);
+            if (lane == 0) red[g * 4 + sub] = l;
+            if (row == 0) misc[g] = m_ref[g];
+          }
+        }
+        bool okv = true;
+        if (wgi == 0 && r.ntiles > 0) {
+          const uint32_t last = it - 1;
+          okv = __all_sync(0xffffffffu, mbar_wait(&pempty[last & 1u], (last >> 1) & 1u, abort_flag));
+          tc_fence_after();
+        }
+        for (int g = 0; g < G; ++g) {
+          named_barrier(1, kEpiThreads);            // red, misc visible; scratch free
+          if (wgi == 0 && sub == 0) {
+            // V accumulator lanes 0 (hi) and 1 (lo) of head g -> olat
+            if (r.ntiles > 0 && okv) {
+              for (int c = 0; c < p.N_v; c += 16) {
+                float v[16];
+                tmem_ld16(tmem_base + p.v_col0 + g * p.N_v + c, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const float o = v[e] + __shfl_down_sync(0xffffffffu, v[e], 1);
+                  if (lane == 0 && c + e < p.r_v) olat[c + e] = o;
+                }
+              }
+            } else {
+              for (int m = lane; m < p.r_v; m += 32) olat[m] = 0.f;
+            }
+          }
+          named_barrier(1, kEpiThreads);            // olat complete
+          const float m_h = r.ntiles > 0 ? misc[g] : -INFINITY;
+          const float l_h = (red[g * 4] + red[g * 4 + 1]) + (red[g * 4 + 2] + red[g * 4 + 3]);
+          const float s_self =
+              p.kappa * ((misc[8 + g * 4] + misc[8 + g * 4 + 1]) + (misc[8 + g * 4 + 2] + misc[8 + g * 4 + 3]));
+          const float M = fmaxf(m_h, s_self);
+          const float a = r.ntiles > 0 ? exp2f(m_h - M) : 0.f, bsf = exp2f(s_self - M);
+          const float inv = 1.f / (l_h * a + bsf);
+          // up-projection: warpgroup hf sums half of the latent dims for output dim d_i
+          const int d_i = et & 127, hf = et >> 7;
+          const int half_r = (p.r_v + 1) / 2, m0 = hf * half_r, m1 = min(p.r_v, m0 + half_r);
+          const size_t bh = (size_t)r.b * p.H + r.hg * G + g;
+          float vs_d = 0.f, mu_d = 0.f;
+          if (hf == 0 && d_i < p.d) {
+            vs_d = __ldg(p.v_self + bh * p.d + d_i);
+            mu_d = __ldg(p.muv_t + (size_t)(r.hg * G + g) * p.d + d_i);
+          }
+          float y = 0.f;
+          if (d_i < p.d) {
+            const float* Wt = p.wupv_t + (size_t)(r.hg * G + g) * p.d * p.r_v + d_i;
+            for (int mb = m0; mb < m1; mb += 16) {
+              float wv[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) wv[e] = mb + e < m1 ? __ldg(Wt + (size_t)(mb + e) * p.d) : 0.f;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) y = fmaf(wv[e], mb + e < m1 ? olat[mb + e] : 0.f, y);
+            }
+          }
+          yh[hf * 128 + d_i] = y;
+          named_barrier(1, kEpiThreads);            // both halves written
+          if (hf == 0 && d_i < p.d)
+            p.out[bh * p.d + d_i] = ((yh[d_i] + yh[128 + d_i]) * a + mu_d * (l_h * a) + vs_d * bsf) * inv;
+        }
+        named_barrier(1, kEpiThreads);              // scratch free for the next item
+      } else if (wgi == 0 && r.ntiles > 0) {
         const size_t bh0 = (size_t)r.b * p.H + r.hg * G;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -984,19 +1076,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         named_barrier(2, 128);
-      } else if (wgi == 0) {
+      } else if (wgi == 0 && !FUSE) {
         // no tiles in this split: empty partial
         const size_t bh0 = (size_t)r.b * p.H + r.hg * G;
         for (int idx = row; idx < G * (2 + p.r_v); idx += 128) {
           const int g = idx / (2 + p.r_v), m = idx % (2 + p.r_v);
           p.partials[((bh0 + g) * p.S + r.s) * (2 + p.r_v) + m] = m == 0 ? -INFINITY : 0.f;
         }
-      }
-      if constexpr (FUSE) if (wgi == 0) {
-        // ---- fused combine: the group has one split, computed right here
-        __threadfence();
-        named_barrier(2, 128);
-        for (int g = 0; g < G; ++g) combine_head(p, r.b, r.hg * G + g, sm + p.comb_off, row, 2);
       }
     }
   }
@@ -1566,8 +1652,8 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst, int nst_v) {
   o += 2 * G * 8 * kTile * 2;
   p.sbuf_off = o;
   o += 2 * (kEpiWG - 1) * G * kTile * 4;
-  p.comb_off = o;                    // fused combine: olat [256], split weights [64], red [8], flag
-  o += (256 + 64 + 8 + 4) * 4;
+  p.comb_off = o;                    // fused finish: olat [256], up-projection halves [256], misc [32]
+  o += (256 + 256 + 32) * 4;
   p.red_off = o;
   o = al(o + G * 4 * 4, 16);
   p.ctx_off = o;
