@@ -312,6 +312,9 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
     unsigned char* __restrict__ ops_bias, int32_t* status, uint32_t* counters, int d_full) {
   constexpr int HALF = D / 2;
   const int NS = d_full > D ? D + 16 : D;      // rows of the images
+  // the partial kernel may start its prologue and latent loads now; it waits for
+  // this grid before it reads the images or the counter
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float2 qc[HALF];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   // the CTA counter of the fused-combine kernels starts every call at zero (this
@@ -609,7 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const ItemRange r = item_range(p, ctx_s, item, false);
         if (r.ntiles == 0) continue;
         if (kside) {
-          // query-absorbed operands of this item into B buffer jn & 1
+          // query-absorbed operands of this item into B buffer jn & 1 (written by the
+          // prep grid, which may still be running when this kernel starts)
+          if (jn == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
           const uint32_t buf = jn & 1u, bph = (jn >> 1) & 1u;
           if (!mbar_wait(&bempty[buf], bph ^ 1u, abort_flag)) break;
           const size_t head0 = (size_t)r.b * p.H + (size_t)r.hg * G;
@@ -1094,6 +1099,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
   if (threadIdx.x == 0) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // prep's counter and status writes
     if (*abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
     if constexpr (FUSE) {
       // with the combine fused in, the last CTA to finish publishes this call's status
@@ -1866,8 +1872,22 @@ cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcPa
     kern = p.fuse_combine ? decode_tc_kernel<D, G, true, NOPE> : decode_tc_kernel<D, G, false, NOPE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, SHARED ? kThreads2 : kThreads, smem, s>>>(mk, mv, p);
-  return cudaGetLastError();
+  if (SHARED || !p.fuse_combine) {
+    kern<<<grid, SHARED ? kThreads2 : kThreads, smem, s>>>(mk, mv, p);
+    return cudaGetLastError();
+  }
+  // one-split per-head plan: programmatic dependent launch after the prep kernel
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
 }
 
 template <int D>
