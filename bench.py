@@ -41,7 +41,7 @@ NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 278.04e6,
 # The same for the full-memory fast path (dominant kernel: full_decode_kernel).
 NCU_TRAFFIC_FULL = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 272.19e6}
 # The same for decoupled RoPE (--d-rope), keyed by (workload, d_rope).
-NCU_TRAFFIC_DECOUPLED = {}
+NCU_TRAFFIC_DECOUPLED = {("perhead_4x_T4_H16_d128_r96_160_B8_n4096", 64): 276.60e6}
 
 
 def parse():
