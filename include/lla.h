@@ -85,8 +85,9 @@ typedef struct lla_cfg {
                        d_rope dims of q and k rotate, as a rotary vector of their own width
                        (pairs (i, i + d_rope/2), angle pos * rope_base^(-2 i / d_rope)),
                        and the other dims form a NoPE content path that decode absorbs into
-                       the query.  Supported: 32 or 64, below d_head, per-head mode, decode
-                       on the tensor-core path; d_rope == d_head is the default RoPE. */
+                       the query.  Supported: 32 or 64, below d_head, decode on the
+                       tensor-core path (per head and LLA-2D); d_rope == d_head is the
+                       default RoPE. */
 } lla_cfg;
 
 /* Last error message of the calling thread ("" if none). Never NULL. */

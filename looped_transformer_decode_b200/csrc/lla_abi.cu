@@ -308,7 +308,7 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
   SplitPlan plan = split_plan(*cfg, B, n_cap);
   if (has_nope(*cfg) && n_cap > 0 && !plan.tensor_cores)
     return fail(LLA_ERR_UNSUPPORTED,
-                "decoupled RoPE (d_rope=%d) runs on the per-head tensor-core path only",
+                "decoupled RoPE (d_rope=%d) runs on the tensor-core path only",
                 cfg->d_rope);
   const size_t ops_at = kWsHeader + align_up(partials_bytes(*cfg, B, plan.splits), 256);
   const size_t counters_at = ops_at + align_up(plan.ops_bytes, 256);

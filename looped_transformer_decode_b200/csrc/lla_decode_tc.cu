@@ -1134,10 +1134,11 @@ constexpr int kEpiWarps2 = kEpiThreads2 / 32;
 constexpr int kThreads2 = 64 + kEpiThreads2 + 64;
 constexpr int kVProdWarp2 = 2 + kEpiWarps2, kVMmaWarp2 = 3 + kEpiWarps2;
 
-template <int D, int HP, bool FUSE>
+template <int D, int HP, bool FUSE, bool NOPE>
 __global__ void __launch_bounds__(kThreads2, 1)
     decode_tc2d_kernel(const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
+  constexpr int NS = D + (NOPE ? 16 : 0);   // score columns per head (see decode_tc_kernel)
   constexpr int HALF = D / 2;
   constexpr int WG_PAIRS = HALF / kEpiWG2;
   static_assert(HP <= kEpiWG2, "one finalizing warpgroup per head");
@@ -1286,7 +1287,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ score MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, D);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, NS);
       const uint32_t sbo_a = 16u * p.box_k;
       const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 0, 0);   // rows alias
       uint32_t it = 0, jn = 0, u = 0;
@@ -1318,7 +1319,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + acc * D;
+            const uint32_t d_tmem = tmem_base + acc * NS;
             const uint32_t b_addr = b_base + g * ops_head_bytes;
             for (int kk = 0; kk < p.K_pad / 16; ++kk) {
               const int kb = (kk * 16) / p.box_k, kin = (kk * 16) % p.box_k;
@@ -1442,11 +1443,16 @@ __global__ void __launch_bounds__(kThreads2, 1)
                              : mbar_wait(&tfull[acc], aph, abort_flag));
           tc_fence_after();
           float uu[WG_COLS];
-          const uint32_t col = tmem_base + lane_addr + acc * D + wgi * WG_COLS;
+          const uint32_t col = tmem_base + lane_addr + acc * NS + wgi * WG_COLS;
 #pragma unroll
           for (int c = 0; c < WG_COLS / 16; ++c) tmem_ld16(col + c * 16, uu + c * 16);
           if constexpr (WG_COLS % 16 != 0)
             tmem_ld8(col + (WG_COLS / 16) * 16, uu + (WG_COLS / 16) * 16);
+          float un[8];
+          un[0] = 0.f;
+          if constexpr (NOPE) {
+            if (wgi == 0) tmem_ld8(tmem_base + lane_addr + acc * NS + D, un);   // NoPE content column
+          }
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
@@ -1457,7 +1463,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
             a0 = ffma2(make_float2(uu[2 * q], uu[2 * q + 1]), ef[q], a0);
             if (q + 1 < WG_PAIRS) a1 = ffma2(make_float2(uu[2 * q + 2], uu[2 * q + 3]), ef[q + 1], a1);
           }
-          sbuf[((par * HP + g) * kEpiWG2 + wgi) * kTile + row] = (a0.x + a0.y) + (a1.x + a1.y);
+          sbuf[((par * HP + g) * kEpiWG2 + wgi) * kTile + row] = (a0.x + a0.y) + (a1.x + a1.y) + un[0];
         }
         if (epi_barrier_or_n<kEpiThreads2>(!ok)) {
           aborted = true;
@@ -1736,7 +1742,6 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   // score columns per head: the rotated dims, plus 16 (the NoPE content column and
   // zero padding) with decoupled RoPE, which only the per-head kernel takes
   const bool nope = has_nope(c);
-  if (nope && c.mode == LLA_MODE_2D) return pl;
   const int D = nope ? rotary_dims(c) + 16 : c.d_head;
   const int forced_g = env_int("LLA_TC_G", 0), forced_nst = env_int("LLA_TC_NST", 0);
   const int N_v = (c.r_v + 15) / 16 * 16;
@@ -1867,7 +1872,7 @@ cudaError_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcPa
                         uint32_t smem, int grid, cudaStream_t s) {
   void (*kern)(CUtensorMap, CUtensorMap, TcParams);
   if constexpr (SHARED)
-    kern = p.fuse_combine ? decode_tc2d_kernel<D, G, true> : decode_tc2d_kernel<D, G, false>;
+    kern = p.fuse_combine ? decode_tc2d_kernel<D, G, true, NOPE> : decode_tc2d_kernel<D, G, false, NOPE>;
   else
     kern = p.fuse_combine ? decode_tc_kernel<D, G, true, NOPE> : decode_tc_kernel<D, G, false, NOPE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1904,14 +1909,17 @@ cudaError_t launch_tc_d(int G, bool shared, const CUtensorMap& mk, const CUtenso
   }
 }
 
-// Decoupled RoPE (per-head kernel only): D is the rotary branch width.
+// Decoupled RoPE: D is the rotary branch width.
 template <int D>
-cudaError_t launch_tc_nope(int G, const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
-                           uint32_t smem, int grid, cudaStream_t s) {
-  switch (G) {
-    case 1: return launch_tc_t<D, 1, false, true>(mk, mv, p, smem, grid, s);
-    case 2: return launch_tc_t<D, 2, false, true>(mk, mv, p, smem, grid, s);
-    case 4: return launch_tc_t<D, 4, false, true>(mk, mv, p, smem, grid, s);
+cudaError_t launch_tc_nope(int G, bool shared, const CUtensorMap& mk, const CUtensorMap& mv,
+                           const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
+  switch (G * 2 + (shared ? 1 : 0)) {
+    case 2: return launch_tc_t<D, 1, false, true>(mk, mv, p, smem, grid, s);
+    case 4: return launch_tc_t<D, 2, false, true>(mk, mv, p, smem, grid, s);
+    case 8: return launch_tc_t<D, 4, false, true>(mk, mv, p, smem, grid, s);
+    case 3: return launch_tc_t<D, 1, true, true>(mk, mv, p, smem, grid, s);
+    case 5: return launch_tc_t<D, 2, true, true>(mk, mv, p, smem, grid, s);
+    case 9: return launch_tc_t<D, 4, true, true>(mk, mv, p, smem, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1974,7 +1982,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.r_v = a.r_v;
   // At least 120 KB so that two CTAs never share an SM (each may hold all of TMEM).
   const int ns = pl.nope ? a.rd + 16 : a.d;   // score columns per head
-  uint32_t smem = pl.shared ? tc2d_layout(p, a.d, pl.G, pl.nst, pl.nst_v, pl.nbuf_b)
+  uint32_t smem = pl.shared ? tc2d_layout(p, ns, pl.G, pl.nst, pl.nst_v, pl.nbuf_b)
                             : tc_layout(p, ns, pl.G, pl.nst, pl.nst_v);
   if (smem < 120u * 1024u) smem = 120u * 1024u;
   p.B = a.B;
@@ -1985,7 +1993,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.n_items = a.B * p.HG * pl.S;
   p.rope_max_pos = a.rope_max_pos;
   p.nacc = pl.nacc;
-  p.acc_cols = pl.shared ? a.d : pl.G * ns;
+  p.acc_cols = pl.shared ? ns : pl.G * ns;
   p.v_col0 = p.nacc * p.acc_cols;
   const int v_cols = pl.shared ? p.m_v * p.n_p : pl.G * p.N_v;
   int cols = 32;
@@ -2045,8 +2053,8 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   cudaError_t e;
   if (pl.nope) {
     switch (a.rd) {
-      case 32: e = launch_tc_nope<32>(pl.G, mk, mv, p, smem, grid, s); break;
-      case 64: e = launch_tc_nope<64>(pl.G, mk, mv, p, smem, grid, s); break;
+      case 32: e = launch_tc_nope<32>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
+      case 64: e = launch_tc_nope<64>(pl.G, pl.shared, mk, mv, p, smem, grid, s); break;
       default: return cudaErrorNotSupported;
     }
   } else {

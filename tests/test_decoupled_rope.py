@@ -5,9 +5,9 @@ first d_rope dims of each head.
 CPU: the oracle pinned to the full-RoPE decode (d_rope = d), to a NoPE attention
 written out by hand (d_rope = 0), to its own absorbed form, and to the
 relative-position property of the rotary branch; host checks of the ABI.
-GPU: the per-head tensor-core decode with d_rope in {32, 64} against the oracle
-(ragged and random-position cases, several splits and one split per head), and
-the refusal of shapes outside that path.
+GPU: the tensor-core decode (per head and LLA-2D) with d_rope in {32, 64} against
+the oracle (ragged and random-position cases, several splits and one split per
+head), and the refusal of the CUDA-core path.
 """
 from __future__ import annotations
 
@@ -154,6 +154,8 @@ DECOUPLED_CASES = [
     (O.Cfg(4, 4, 128, 16, 32), 32, [200, 64], "arange"),
     (O.Cfg(2, 2, 96, 32, 48), 64, [130, 7], "random"),
     (O.Cfg(2, 4, 64, 24, 40), 32, [100], "random"),
+    (O.Cfg(2, 4, 128, 64, 128, O.MODE_2D), 64, [260, 100], "random"),   # LLA-2D
+    (O.Cfg(2, 8, 64, 32, 48, O.MODE_2D), 32, [200, 1, 129], "arange"),
 ]
 
 
@@ -206,14 +208,9 @@ def test_decoupled_rope_outside_the_tensor_core_path_is_refused(monkeypatch):
 
     import looped_transformer_decode_b200 as lla
     from cases import decode_case
-    cfg = O.Cfg(2, 2, 64, 16, 16)
-    case = decode_case(cfg, 1, 40, seed=960, codec="random")
-    monkeypatch.setenv("LLA_DECODE_PATH", "cuda_core")
-    with pytest.raises(lla.LLAError):
-        _run_decoupled(case, 32, 0)
-    cfg2 = O.Cfg(2, 4, 64, 16, 16, O.MODE_2D)
-    case2 = decode_case(cfg2, 1, 40, seed=961, codec="random")
-    monkeypatch.delenv("LLA_DECODE_PATH")
-    with pytest.raises(lla.LLAError):
-        _run_decoupled(case2, 32, 0)
+    for cfg in (O.Cfg(2, 2, 64, 16, 16), O.Cfg(2, 4, 64, 16, 16, O.MODE_2D)):
+        case = decode_case(cfg, 1, 40, seed=960, codec="random")
+        monkeypatch.setenv("LLA_DECODE_PATH", "cuda_core")
+        with pytest.raises(lla.LLAError):
+            _run_decoupled(case, 32, 0)
     torch.cuda.synchronize()
