@@ -60,6 +60,9 @@ def parse():
                    help="latent: decode over the latent cache (rebuild on read); full: the "
                         "full-memory fast path (K/V rebuilt once per token into a full bf16 "
                         "cache per loop, ordinary attention)")
+    p.add_argument("--graph", action="store_true",
+                   help="capture a step (every layer's decode at each loop, then the encode "
+                        "of the finished tokens) as CUDA graphs and time their replays")
     p.add_argument("--d-rope", type=int, default=0,
                    help="decoupled RoPE: rotate only the first D_ROPE dims of each head and "
                         "absorb the rest into a NoPE content path (32 or 64; 0 = whole head)")
@@ -269,7 +272,7 @@ def run_step_full(lla, w, st, events=None):
     the new tokens and rebuild their rows into every loop's cache."""
     if st.get("flush") is not None:
         st["flush"].add_(1)
-    for t in w.loops:
+    for t in ([] if st.get("skip_decode") else w.loops):
         for L in st["layers"]:
             if events is not None:
                 events[0].append(_event())
@@ -278,7 +281,7 @@ def run_step_full(lla, w, st, events=None):
                                  L["v_self"], L["q_pos"], kf, vf, out=st["out"], ws=st["fws"])
             if events is not None:
                 events[1].append(_event())
-    for L in st["layers"]:
+    for L in ([] if st.get("skip_append") else st["layers"]):
         if events is not None:
             events[2].append(_event())
         lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
@@ -290,12 +293,46 @@ def run_step_full(lla, w, st, events=None):
             events[3].append(_event())
 
 
+def capture_step_graphs(lla, w, st):
+    """The step as two CUDA graphs: every layer's decode at each loop, then the
+    encode (and, on the full-memory path, the row rebuild) of the finished tokens."""
+    import torch
+
+    flush = st.pop("flush", None)               # the L2 flush stays outside the graphs
+    g_dec, g_enc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    dec_only = dict(st, skip_append=True)
+    with torch.cuda.graph(g_dec):
+        run_step(lla, w, dec_only)
+    enc_only = dict(st, skip_decode=True)
+    with torch.cuda.graph(g_enc):
+        run_step(lla, w, enc_only)
+    torch.cuda.synchronize()
+    return {"dec": g_dec, "enc": g_enc, "flush": flush}
+
+
+def replay_step_graphs(st, graphs, events, n_dec, n_enc):
+    """One timed step from the captured graphs; the per-call times are the graph
+    times divided by the calls each graph holds."""
+    if graphs["flush"] is not None:
+        graphs["flush"].add_(1)
+    e = [_event() for _ in range(3)]
+    e[0].record()
+    graphs["dec"].replay()
+    e[1].record()
+    graphs["enc"].replay()
+    e[2].record()
+    events[0].append((e[0], n_dec))
+    events[1].append((e[1], n_dec))
+    events[2].append((e[1], n_enc))
+    events[3].append((e[2], n_enc))
+
+
 def run_step(lla, w, st, events=None):
     if st.get("full_path"):
         return run_step_full(lla, w, st, events)
     if st.get("flush") is not None:
         st["flush"].add_(1)                       # working set below L2: evict it first
-    for t in w.loops:
+    for t in ([] if st.get("skip_decode") else w.loops):
         for L in st["layers"]:
             if events is not None:
                 events[0].append(_event())
@@ -304,7 +341,7 @@ def run_step(lla, w, st, events=None):
                             L["c_v"], out=st["out"], ws=st["ws"])
             if events is not None:
                 events[1].append(_event())
-    for L in st["layers"]:
+    for L in ([] if st.get("skip_append") else st["layers"]):
         if events is not None:
             events[2].append(_event())
         lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
@@ -428,21 +465,30 @@ def run_gpu(args):
             break
 
     ev_pairs = ([], [], [], [])
+    graphs = capture_step_graphs(lla, w, st) if args.graph else None
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier_sync(dist_on)
     if clocks:
         clocks.mark_start()
     start.record()
     for _ in range(args.steps):
-        run_step(lla, w, st, ev_pairs)
+        if graphs:
+            replay_step_graphs(st, graphs, ev_pairs, len(w.loops) * w.layers, w.layers)
+        else:
+            run_step(lla, w, st, ev_pairs)
     stop.record()
     barrier_sync(dist_on)
     if clocks:
         clocks.mark_stop()
     ms = start.elapsed_time(stop)
     clk = clocks.stop() if clocks else None
-    dec_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[0], ev_pairs[1])]
-    enc_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[2], ev_pairs[3])]
+    if graphs:
+        # graph replays: per-call times are the graph times over the calls they hold
+        dec_ms = [a[0].elapsed_time(b[0]) / a[1] for a, b in zip(ev_pairs[0], ev_pairs[1])]
+        enc_ms = [a[0].elapsed_time(b[0]) / a[1] for a, b in zip(ev_pairs[2], ev_pairs[3])]
+    else:
+        dec_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[0], ev_pairs[1])]
+        enc_ms = [a.elapsed_time(b) for a, b in zip(ev_pairs[2], ev_pairs[3])]
     status = lla.decode_status(st["fws"] if full else st["ws"])
     if status:
         raise RuntimeError(f"decode reported device status bits {status}")
@@ -496,7 +542,9 @@ def run_gpu(args):
                    "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
                    "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
                    "evict": list(evict) if evict else None, "attended_context": n_ctx,
-                   "path": args.path, "d_rope": args.d_rope or None, "l2": l2_note},
+                   "path": args.path, "d_rope": args.d_rope or None,
+                   "schedule": "cuda graph per step" if args.graph else "eager launches",
+                   "l2": l2_note},
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
         "roofline": {"bound": "hbm", "kernel": kname,
