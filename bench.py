@@ -60,9 +60,10 @@ def parse():
                    help="latent: decode over the latent cache (rebuild on read); full: the "
                         "full-memory fast path (K/V rebuilt once per token into a full bf16 "
                         "cache per loop, ordinary attention)")
-    p.add_argument("--graph", action="store_true",
-                   help="capture a step (every layer's decode at each loop, then the encode "
-                        "of the finished tokens) as CUDA graphs and time their replays")
+    p.add_argument("--eager", action="store_true",
+                   help="launch every call of a timed step from the host; by default a step "
+                        "(every layer's decode at each loop, then the encode of the finished "
+                        "tokens) is captured once as CUDA graphs and the replays are timed")
     p.add_argument("--d-rope", type=int, default=0,
                    help="decoupled RoPE: rotate only the first D_ROPE dims of each head and "
                         "absorb the rest into a NoPE content path (32 or 64; 0 = whole head)")
@@ -465,7 +466,7 @@ def run_gpu(args):
             break
 
     ev_pairs = ([], [], [], [])
-    graphs = capture_step_graphs(lla, w, st) if args.graph else None
+    graphs = None if args.eager else capture_step_graphs(lla, w, st)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier_sync(dist_on)
     if clocks:
@@ -517,7 +518,7 @@ def run_gpu(args):
     else:
         unit_bytes, unit_ms = dec_bytes(w, n_ctx), dec_avg
         kname = ("lla_full_decode_attn (full_decode_kernel [+ combine])" if full
-                 else "lla_decode_attn (prep + partial + combine)")
+                 else "lla_decode_attn (prep + partial kernel [+ combine])")
     achieved = unit_bytes / (unit_ms * 1e-3) / 1e9
 
     e2e = None
@@ -543,7 +544,7 @@ def run_gpu(args):
                    "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
                    "evict": list(evict) if evict else None, "attended_context": n_ctx,
                    "path": args.path, "d_rope": args.d_rope or None,
-                   "schedule": "cuda graph per step" if args.graph else "eager launches",
+                   "schedule": "eager launches" if args.eager else "cuda graphs per step",
                    "l2": l2_note},
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
