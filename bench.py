@@ -358,13 +358,27 @@ def _event():
     return e
 
 
-def barrier_sync(dist_on):
+def barrier_sync(dist_on, cuda=True):
     import torch
     import torch.distributed as dist
 
     if dist_on:
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
+
+
+def over_ranks(values, op, device, dist_on):
+    """Element-wise max ("max") or min ("min") of a list of floats over all ranks
+    (every rank takes part; identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist_on:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.MIN)
+    return [float(v) for v in t]
 
 
 def cpu_baseline_sample(w, seconds: float, loops=None, d_rope=0):
@@ -458,10 +472,7 @@ def run_gpu(args):
         run_step(lla, w, st)
         torch.cuda.synchronize()
         done = 1.0 if (clocks is None or clocks.lines() >= 2 or time.time() - t_w > 5.0) else 0.0
-        if dist_on:
-            flag = torch.tensor([done], device=device)
-            dist.all_reduce(flag, op=dist.ReduceOp.MIN)
-            done = float(flag)
+        done = over_ranks([done], "min", device, dist_on)[0]
         if done:
             break
 
@@ -493,12 +504,9 @@ def run_gpu(args):
     status = lla.decode_status(st["fws"] if full else st["ws"])
     if status:
         raise RuntimeError(f"decode reported device status bits {status}")
-    if dist_on:
-        tt = torch.tensor([ms, float(np.mean(dec_ms)), float(np.mean(enc_ms))], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, dec_avg, enc_avg = float(tt[0]), float(tt[1]), float(tt[2])
-    else:
-        dec_avg, enc_avg = float(np.mean(dec_ms)), float(np.mean(enc_ms))
+    # the job's time is the slowest rank's
+    ms, dec_avg, enc_avg = over_ranks([ms, np.mean(dec_ms), np.mean(enc_ms)], "max", device,
+                                      dist_on)
 
     append_bytes = encode_bytes(w, w.encode_tokens)
     if full:
@@ -651,11 +659,7 @@ def run_e2e(lla, w, st, args, dist_on, world, n_ctx):
     e.record()
     barrier_sync(dist_on)
     ms = s.elapsed_time(e) / steps
-    if dist_on:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=st["out"].device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt[0])
+    ms = over_ranks([ms], "max", st["out"].device, dist_on)[0]
     per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, n_ctx)
                       + w.layers * encode_bytes(w, w.encode_tokens))
     return {"value": round(world * per_step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
