@@ -1,25 +1,28 @@
 // LLA decode attention on the 5th-generation tensor cores (sm_100a), per head and
 // LLA-2D.  In LLA-2D every head reads the same latent row (close reading §二.6),
-// so the head offset into the latent is zero and a head group's tiles repeat the
-// same bytes, which L2 serves after the first read.
+// so a work item's heads share each latent tile.
 //
 // Same arithmetic as the CUDA-core kernel (query folded into the K
-// up-projection, RoPE as a complex product with the fp64-built table, base-2
-// online softmax, V summed in latent space), reorganised for B200:
+// up-projection, RoPE as a complex product, base-2 online softmax, V summed in
+// latent space), organised for B200:
 //
+//   * decode_prep_kernel builds, per (b, h), the query-absorbed score operand
+//     A~ = kappa conj(q~) W~ (and the bias M~, bf16 hi + lo) as the byte image of
+//     the MMA's shared-memory operand; with decoupled RoPE it also writes the
+//     NoPE content row;
 //   * persistent CTAs, one per SM, walk a list of work items (sequence b, group
-//     of G heads, context split s); the split partials feed the combine pass;
-//   * warp 0 streams 128-token tiles of c_k and c_v with TMA into an NST-deep
-//     shared-memory ring (c_k tiles land in the swizzled K-major layout the
-//     tensor core reads);
-//   * warp 1 issues tcgen05.mma: U[128 x d] = C_k[128 x r_k] * A~^T[r_k x d] per
-//     head, plus one K=16 MMA with a ones column that adds the per-column bias
-//     M~ (split into bf16 hi + lo), accumulating in fp32 in TMEM;
-//   * warps 2..9 (two warpgroups, each owning half of the RoPE pairs of every
-//     token row) read U from TMEM, form s_j = sum_i Re(U_ji e^{i p_j theta_i}),
-//     run the online softmax, and accumulate sum_j p_j c_v,j from the staged c_v
-//     tile; between items they rebuild A~ and M~ for the next (b, heads) in
-//     shared memory.
+//     of heads, context split s); a TMA producer warp streams 128-token c_k tiles
+//     into a swizzled K-major ring (and each item's operand images with one bulk
+//     copy), another the c_v tiles into an MN-major ring;
+//   * one warp issues the score tcgen05.mma U = C_k A~^T (+ the bias through a
+//     ones column) into fp32 TMEM; the epilogue warpgroups read U, turn the RoPE
+//     pairs at each token's position (complex factors advanced tile to tile),
+//     run the online softmax and write the weights as bf16 hi + lo rows;
+//   * another warp issues the V MMAs that accumulate sum_j p_j c_v,j in TMEM
+//     (per head: P x C_v; LLA-2D: transposed, C_v^T P^T for all heads at once);
+//   * with one split per head group the item is finished in the kernel (merge
+//     with the in-flight token, W_up,v up-projection); otherwise split partials
+//     go to decode_combine_kernel.
 // The close reading §二.3 fixes the order (rebuild K, then RoPE at its
 // position); folding q into W_up and RoPE into a complex dot product changes
 // only the order of the same sums.
