@@ -10,7 +10,8 @@ Pages this follows (cited by page title and section):
 * [CR]  "Looped Latent Attention: 跨循环 KV 压缩精读" (cc.laoqi.cc close reading of
         arXiv 2607.15456v2).  §二.1 symbol table, §二.2 eq. (4) and its worked
         example, §二.3 pre-RoPE compression, §二.4 SVD initialisation,
-        §二.6 LLA-2D, §四.9 Table 5 (serving).
+        §二.6 LLA-2D, §四.9 Table 5 (serving; the full-memory fast path),
+        §四.10 Table 9 and Appendix J (eviction budgets; decoupled RoPE).
 * [GS]  "Looped Latent Attention: Cross-Loop KV Compression for Looped
         Transformers" (gist.science explainer), "Technisches Resümee":
         "Kernmechanismus" (encode / loop-specific decode formulas, LLA-2D),
@@ -27,7 +28,10 @@ Conventions (row vectors throughout, as on [GS] Kernmechanismus):
 
 Readings where the pages are silent are listed in the design notes; the ones
 that change arithmetic are restated next to the function that takes them.
-Every function here is pinned by ``tests/test_oracle_pins.py``.
+Every function here is pinned: the codec, bookkeeping, RoPE and decode by
+``tests/test_oracle_pins.py``, eviction by ``tests/test_evict.py``, the
+full-memory path by ``tests/test_full_memory.py`` and decoupled RoPE by
+``tests/test_decoupled_rope.py`` (their CPU tests).
 """
 from __future__ import annotations
 
