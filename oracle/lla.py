@@ -26,8 +26,8 @@ Conventions (row vectors throughout, as on [GS] Kernmechanismus):
   decode    x^_t = c W_up,t^T + mu_t,           W_up,t in R^{d x r}
   RoPE      split-half: pair (i, i + d/2) rotated by angle pos * base^(-2i/d).
 
-Readings where the pages are silent are listed in the design notes; the ones
-that change arithmetic are restated next to the function that takes them.
+Where the pages are silent, the reading taken is stated next to the function
+that takes it.
 Every function here is pinned: the codec, bookkeeping, RoPE and decode by
 ``tests/test_oracle_pins.py``, eviction by ``tests/test_evict.py``, the
 full-memory path by ``tests/test_full_memory.py`` and decoupled RoPE by
