@@ -9,8 +9,6 @@ from __future__ import annotations
 import os
 import socket
 
-import pytest
-
 
 def _free_port() -> int:
     with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:

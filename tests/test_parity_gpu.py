@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     import looped_transformer_decode_b200 as lla
-    from gpu_util import DeviceCase, bf16_tensor, f32_tensor, i32_tensor, lib_cfg, pack
+    from gpu_util import DeviceCase, bf16_tensor, i32_tensor, lib_cfg, pack
 
 
 # ----------------------------------------------------------------------------- RoPE table
