@@ -93,7 +93,8 @@ typedef struct lla_cfg {
 /* Last error message of the calling thread ("" if none). Never NULL. */
 const char* lla_last_error(void);
 
-/* Library version string. */
+/* Library version string ("lla-b200 <major>.<minor> ..."); 0.2 added lla_cfg.d_rope,
+ * the full-memory fast path and the eviction calls. */
 const char* lla_version(void);
 
 /* ------------------------------------------------------------------------ */

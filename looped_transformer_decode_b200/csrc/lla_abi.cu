@@ -153,7 +153,7 @@ extern "C" {
 
 const char* lla_last_error(void) { return g_err.c_str(); }
 
-const char* lla_version(void) { return "lla-b200 0.1 (sm_100a)"; }
+const char* lla_version(void) { return "lla-b200 0.2 (sm_100a)"; }
 
 int lla_ratio(const lla_cfg* cfg, int64_t* num, int64_t* den) {
   int e = check_cfg(cfg);
