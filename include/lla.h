@@ -236,10 +236,13 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
  * in a fixed device array of 8 MiB (8388608 bytes) that the library holds on
  * every GPU where it is loaded, until the process exits.
  *   - Shapes whose workspace (lla_decode_workspace_bytes) exceeds 8 MiB are
- *     rejected with LLA_ERR_TOO_SMALL before anything is enqueued.
+ *     rejected with LLA_ERR_TOO_SMALL, and every argument lla_decode_attn checks
+ *     is checked, before anything is enqueued: a rejected call leaves the array
+ *     and status_out untouched.  B == 0 enqueues nothing.
  *   - The first call on a device looks up the array's device address with that
  *     device current (cudaGetSymbolAddress); make that first call before any
- *     stream capture.  Later calls reuse the address.
+ *     stream capture.  Later calls reuse the address while the device keeps the
+ *     same CUDA context, and look it up again after a device reset.
  *   - All calls share the one array and it keeps the last call's contents.  Each
  *     call clears the status words it needs; calls that overlap on the GPU (on
  *     different streams, or from different threads) race on the array and must

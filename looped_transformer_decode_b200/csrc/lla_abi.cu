@@ -103,6 +103,17 @@ PackedLayout packed_layout(const lla_cfg& c) {
   return L;
 }
 
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0) {
+    cudaGetLastError();   // a failed query leaves an error behind; clear it
+    return 148;
+  }
+  return sms;
+}
+
 SplitPlan split_plan(const lla_cfg& c, int B, int n_cap) {
   SplitPlan p{};
   p.n_tiles = (n_cap + kTile - 1) / kTile;
@@ -120,15 +131,47 @@ SplitPlan split_plan(const lla_cfg& c, int B, int n_cap) {
     p.ops_bytes = ops;
     return p;
   }
-  // Aim for about four resident CTAs per SM on a 148-SM part.
+  // Aim for about four resident CTAs per SM.
   const long long units = (long long)B * c.H;
-  long long want = (4 * 148 + units - 1) / units;
+  long long want = (4 * sm_count() + units - 1) / units;
   if (want < 1) want = 1;
   if (want > kMaxSplits) want = kMaxSplits;
   if (want > p.n_tiles) want = p.n_tiles;
   p.tiles_per_split = (p.n_tiles + (int)want - 1) / (int)want;
   p.splits = (p.n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
   return p;
+}
+
+int decode_check_args(const lla_cfg* cfg, const void* packed, const void* rope_table,
+                      int32_t rope_max_pos, int32_t t, int32_t B, int32_t n_cap,
+                      const int32_t* ctx_len, const float* q, const float* k_self,
+                      const float* v_self, const int32_t* positions, const int32_t* q_pos,
+                      const uint16_t* c_k, const uint16_t* c_v, const float* out) {
+  int e = check_cfg(cfg);
+  if (e) return e;
+  if (t < 0 || t >= cfg->T) return fail(LLA_ERR_INVALID, "t=%d outside [0, T=%d)", t, cfg->T);
+  if (B < 0 || n_cap < 0) return fail(LLA_ERR_INVALID, "B and n_cap must be >= 0");
+  if (B > 65535) return fail(LLA_ERR_UNSUPPORTED, "B=%d above 65535", B);
+  if (rope_max_pos < 1) return fail(LLA_ERR_INVALID, "rope_max_pos must be >= 1");
+  if ((long long)B * n_cap > (1LL << 40)) return fail(LLA_ERR_UNSUPPORTED, "B * n_cap too large");
+  if (B == 0) return ok();
+  const void* ptrs[] = {packed, rope_table, ctx_len, q, k_self, v_self, q_pos, out};
+  for (const void* p : ptrs) {
+    if (!p) return fail(LLA_ERR_INVALID, "lla_decode_attn: NULL pointer argument");
+    if (!aligned16(p)) return fail(LLA_ERR_INVALID, "lla_decode_attn: pointer not 16-byte aligned");
+  }
+  if (n_cap > 0) {
+    const void* hist[] = {positions, c_k, c_v};
+    for (const void* p : hist) {
+      if (!p) return fail(LLA_ERR_INVALID, "lla_decode_attn: NULL history pointer");
+      if (!aligned16(p)) return fail(LLA_ERR_INVALID, "lla_decode_attn: history pointer misaligned");
+    }
+  }
+  if (has_nope(*cfg) && n_cap > 0 && !split_plan(*cfg, B, n_cap).tensor_cores)
+    return fail(LLA_ERR_UNSUPPORTED,
+                "decoupled RoPE (d_rope=%d) runs on the tensor-core path only",
+                cfg->d_rope);
+  return ok();
 }
 
 size_t partials_bytes(const lla_cfg& c, int B, int S) {
@@ -285,31 +328,13 @@ int lla_decode_attn(const lla_cfg* cfg, const void* packed, const void* rope_tab
                     const float* v_self, const int32_t* positions, const int32_t* q_pos,
                     const uint16_t* c_k, const uint16_t* c_v, float* out, void* ws,
                     size_t ws_bytes, void* stream) {
-  int e = check_cfg(cfg);
+  int e = lla::decode_check_args(cfg, packed, rope_table, rope_max_pos, t, B, n_cap, ctx_len, q,
+                                 k_self, v_self, positions, q_pos, c_k, c_v, out);
   if (e) return e;
-  if (t < 0 || t >= cfg->T) return fail(LLA_ERR_INVALID, "t=%d outside [0, T=%d)", t, cfg->T);
-  if (B < 0 || n_cap < 0) return fail(LLA_ERR_INVALID, "B and n_cap must be >= 0");
-  if (B > 65535) return fail(LLA_ERR_UNSUPPORTED, "B=%d above 65535", B);
-  if (rope_max_pos < 1) return fail(LLA_ERR_INVALID, "rope_max_pos must be >= 1");
-  if ((long long)B * n_cap > (1LL << 40)) return fail(LLA_ERR_UNSUPPORTED, "B * n_cap too large");
   if (B == 0) return ok();
-  const void* ptrs[] = {packed, rope_table, ctx_len, q, k_self, v_self, q_pos, out, ws};
-  for (const void* p : ptrs) {
-    if (!p) return fail(LLA_ERR_INVALID, "lla_decode_attn: NULL pointer argument");
-    if (!aligned16(p)) return fail(LLA_ERR_INVALID, "lla_decode_attn: pointer not 16-byte aligned");
-  }
-  if (n_cap > 0) {
-    const void* hist[] = {positions, c_k, c_v};
-    for (const void* p : hist) {
-      if (!p) return fail(LLA_ERR_INVALID, "lla_decode_attn: NULL history pointer");
-      if (!aligned16(p)) return fail(LLA_ERR_INVALID, "lla_decode_attn: history pointer misaligned");
-    }
-  }
+  if (!ws) return fail(LLA_ERR_INVALID, "lla_decode_attn: NULL pointer argument");
+  if (!aligned16(ws)) return fail(LLA_ERR_INVALID, "lla_decode_attn: pointer not 16-byte aligned");
   SplitPlan plan = split_plan(*cfg, B, n_cap);
-  if (has_nope(*cfg) && n_cap > 0 && !plan.tensor_cores)
-    return fail(LLA_ERR_UNSUPPORTED,
-                "decoupled RoPE (d_rope=%d) runs on the tensor-core path only",
-                cfg->d_rope);
   const size_t ops_at = kWsHeader + align_up(partials_bytes(*cfg, B, plan.splits), 256);
   const size_t counters_at = ops_at + align_up(plan.ops_bytes, 256);
   size_t need = counters_at + (plan.tensor_cores ? align_up(((size_t)B * cfg->H + 1) * 4, 256) : 0);

@@ -1822,15 +1822,17 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   pl.nst_v = best_nst_v;
   pl.nacc = best_nacc;
   // Context splits: the split count S minimises the busiest CTA's cost over a
-  // 148-SM grid of persistent CTAs, where items are dealt round-robin and each
+  // grid of one persistent CTA per SM, where items are dealt round-robin and each
   // item costs its tiles plus a fixed start/finish charge (operand hand-over, the
   // V-accumulator drain and the partial write, about 1.6 tiles of time measured on
   // the per-head 4x workload); more than one split also pays the combine pass.
   const int n_tiles = (n_cap + kTile - 1) / kTile;
   const long long units = (long long)B * (c.H / pl.G);
-  const int grid = 148;
+  const int grid = sm_count();
   constexpr double kItemCost = 1.6, kCombineCost = 0.5;   // in tiles
-  const int forced_s = env_int("LLA_TC_SPLITS", 0);
+  // a forced split count obeys the same bounds as a planned one: the combine merges
+  // at most kMaxSplits partials per head, and a split needs at least one tile
+  const int forced_s = std::min(env_int("LLA_TC_SPLITS", 0), std::min(kMaxSplits, n_tiles));
   int s_max = (int)std::max<long long>(1, (4 * grid + units - 1) / units);
   s_max = std::min(std::min(s_max, kMaxSplits), n_tiles);
   double best_cost = 1e300;
@@ -2047,9 +2049,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
                 : p.cvb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                               : CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorNotSupported;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   cudaError_t pe = launch_prep(a, p, s);
   if (pe != cudaSuccess) return pe;
   const int grid = p.n_items < sms ? p.n_items : sms;

@@ -336,9 +336,7 @@ cudaError_t launch_encode_tc(const lla_cfg& c, const PackedLayout& L, const char
   p.nchunks = L.W / p.kc;
   const int n_k = (c.r_k + 15) / 16 * 16, n_v = (c.r_v + 15) / 16 * 16;
   const int n_max = n_k > n_v ? n_k : n_v;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   // Two CTAs per SM when each can hold two accumulators in half of TMEM.
   int cps = 2 * n_max <= (int)kEncTmemCols / 2 ? 2 : 1;
   const char* cps_env = std::getenv("LLA_ENC_CPS");

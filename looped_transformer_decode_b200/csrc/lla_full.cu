@@ -553,7 +553,7 @@ FullPlan full_plan(const lla_cfg& c, int B, int n_cap) {
   FullPlan pl;
   const int D = c.d_head;
   const int per_sm = D % 64 == 0 ? 1 : 2;
-  pl.grid_max = 148 * per_sm;
+  pl.grid_max = sm_count() * per_sm;
   const int n_tiles = std::max(1, (n_cap + kFullTile - 1) / kFullTile);
   const long long units = (long long)B * c.H;
   if (units <= 0) return pl;

@@ -18,6 +18,10 @@ constexpr int kMaxSplits = 64;      // context splits per (b, h) at most
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// SMs of the current device, which sizes every persistent grid and split plan.
+// Without a usable device (host-only use of the sizing calls) a B200's 148.
+int sm_count();
+
 // Offsets (bytes) of each section of the packed codec buffer.
 //   wup_k      fp32 [T][H][d][r]      loop-t, head-h up-projection W_up,k,t,h (d x r)
 //   wup_v      fp32 [T][H][r][d]      W_up,v,t,h transposed (read column-wise by the combine)
@@ -59,6 +63,15 @@ struct SplitPlan {
 };
 SplitPlan split_plan(const lla_cfg& c, int B, int n_cap);
 size_t partials_bytes(const lla_cfg& c, int B, int S);
+
+// Every host check lla_decode_attn makes before it enqueues work, except those of
+// the workspace.  Returns LLA_OK (also for B == 0, which enqueues nothing), or the
+// error code with lla_last_error() set.
+int decode_check_args(const lla_cfg* cfg, const void* packed, const void* rope_table,
+                      int32_t rope_max_pos, int32_t t, int32_t B, int32_t n_cap,
+                      const int32_t* ctx_len, const float* q, const float* k_self,
+                      const float* v_self, const int32_t* positions, const int32_t* q_pos,
+                      const uint16_t* c_k, const uint16_t* c_v, const float* out);
 
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_rope_table(const lla_cfg& c, int max_pos, float2* table, cudaStream_t s);

@@ -7,6 +7,9 @@
 // fixed.  lla_decode_attn_noalloc serves them: it runs the same kernels as
 // lla_decode_attn, with the split-context partials and status words held in a
 // fixed-size array that this library places in device memory when it is loaded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "lla_internal.cuh"
@@ -22,10 +25,38 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};   // context the address belongs to
+
+// Identifier of the calling thread's current CUDA context (0 when it cannot be
+// read).  A device reset or a released and re-created primary context reloads the
+// library's module, and the array may then sit at another address.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with that device current, and cached.
+// array's name is only a host-side stand-in, so the address is looked up with that
+// device current: once per device and context (the first call there), and again
+// whenever the device's context has changed since.
 int scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -35,8 +66,9 @@ int scratch_address(void** out) {
   if (dev < 0 || dev >= kMaxDevices)
     return lla::set_error(LLA_ERR_UNSUPPORTED, "lla_decode_attn_noalloc: device %d above %d", dev,
                           kMaxDevices - 1);
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (!g_scratch_addr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
@@ -44,6 +76,8 @@ int scratch_address(void** out) {
                             "lla_decode_attn_noalloc: cudaGetSymbolAddress failed: %s",
                             cudaGetErrorString(e));
     g_scratch_addr[dev] = p;
+    // read again: the lookup above may have created the primary context
+    g_scratch_ctx[dev] = ctx ? ctx : current_context_id();
   }
   *out = g_scratch_addr[dev];
   return LLA_OK;
@@ -71,6 +105,12 @@ extern "C" int lla_decode_attn_noalloc(const lla_cfg* cfg, const void* packed,
                           need, kNoAllocScratchBytes);
   if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u))
     return lla::set_error(LLA_ERR_INVALID, "lla_decode_attn_noalloc: status_out misaligned");
+  // Every other check of lla_decode_attn, before anything is enqueued: a rejected
+  // call leaves the array (and the last call's status word) as it was.
+  rc = lla::decode_check_args(cfg, packed, rope_table, rope_max_pos, t, B, n_cap, ctx_len, q,
+                              k_self, v_self, positions, q_pos, c_k, c_v, out);
+  if (rc != LLA_OK) return rc;
+  if (B == 0) return LLA_OK;   // nothing to compute; status_out is not written
   void* ws = nullptr;
   rc = scratch_address(&ws);
   if (rc != LLA_OK) return rc;

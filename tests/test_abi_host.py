@@ -135,3 +135,30 @@ def test_decode_plans_of_the_bench_workloads():
     assert lla.decode_launches(lla.Cfg(4, 16, 128, 64, 128, lla.MODE_2D), 512, 4097) == 2
     assert lla.decode_launches(lla.Cfg(32, 8, 96, 64, 128), 16, 32769) == 2
     assert lla.decode_launches(lla.Cfg(4, 16, 128, 96, 160), 1, 4097) == 3
+
+
+def test_forced_split_count_is_clamped(monkeypatch):
+    """LLA_TC_SPLITS obeys the planner's bounds: at most 64 splits per head (the
+    combine's limit) and at most one per 128-token tile.  The workspace holds the
+    split partials [B][H][S][2 + r_v] fp32, so its size shows the S in use."""
+    cfg = lla.Cfg(4, 2, 64, 16, 32)
+    B, n_cap = 1, 32768                      # 256 tiles
+    c = ctypes.byref(cfg.c())
+
+    def partial_bytes(splits):
+        monkeypatch.setenv("LLA_TC_SPLITS", str(splits))
+        return lla.lib.lla_decode_workspace_bytes(c, B, n_cap)
+
+    per_split = B * cfg.H * (2 + cfg.r_v) * 4
+    at64 = partial_bytes(64)
+    assert partial_bytes(100) == at64 == partial_bytes(1000)
+    assert partial_bytes(32) < at64
+    # 64 splits of four tiles each: exactly 64 partials per head (256-byte sections)
+    base = partial_bytes(1)
+    assert at64 - base >= 63 * per_split - 256
+    assert at64 - base <= 63 * per_split + 256
+    # a short history: never more splits than tiles
+    monkeypatch.setenv("LLA_TC_SPLITS", "64")
+    short = lla.lib.lla_decode_workspace_bytes(c, B, 300)    # 3 tiles
+    monkeypatch.setenv("LLA_TC_SPLITS", "3")
+    assert short == lla.lib.lla_decode_workspace_bytes(c, B, 300)

@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 
 import oracle as O
-from cases import ATTN_TOL, decode_case, rel_err
+from cases import ATTN_TOL, decode_case, expected, rel_err
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -49,7 +49,51 @@ def test_noalloc_matches_workspace_entry_point_twice():
         got = _noalloc(dev, t, out, status)
         assert np.isfinite(got).all()
         assert rel_err(got, want).max() <= ATTN_TOL
+        # and element by element against the float64 oracle
+        assert rel_err(got, expected(case, t)).max() <= ATTN_TOL
         assert int(status.item()) == 0
+
+
+def test_noalloc_reports_then_clears_device_status():
+    """A device-side range problem reaches status_out, and the next valid call,
+    which shares the same array, reports a clean status again."""
+    cfg = O.Cfg(4, 2, 64, 16, 32)
+    case = decode_case(cfg, 2, 300, seed=77)
+    dev = DeviceCase(case, rope_max_pos=301)
+    out = torch.empty((case.B, cfg.H, cfg.d), dtype=torch.float32, device="cuda")
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    good_qpos = dev.q_pos
+    bad = case.q_pos.copy()
+    bad[1] = 5000                                      # outside the 301-entry RoPE table
+    dev.q_pos = torch.from_numpy(bad.astype(np.int32)).cuda()
+    got = _noalloc(dev, 0, out, status)
+    assert np.isfinite(got).all()
+    assert int(status.item()) & lla.STATUS_POSITION_RANGE
+    dev.q_pos = good_qpos
+    got = _noalloc(dev, 2, out, status)
+    assert int(status.item()) == 0
+    assert rel_err(got, dev.decode(2)).max() <= ATTN_TOL
+    assert rel_err(got, expected(case, 2)).max() <= ATTN_TOL
+
+
+def test_noalloc_rejected_call_enqueues_nothing():
+    """Arguments that lla_decode_attn rejects are rejected before anything is
+    enqueued, so status_out keeps the last call's word."""
+    cfg = O.Cfg(4, 2, 64, 16, 32)
+    case = decode_case(cfg, 1, 200, seed=78)
+    dev = DeviceCase(case)
+    out = torch.empty((case.B, cfg.H, cfg.d), dtype=torch.float32, device="cuda")
+    status = torch.full((1,), 12345, dtype=torch.int32, device="cuda")
+    p = lambda x: ctypes.c_void_p(x.data_ptr())  # noqa: E731
+    ks = f32_tensor(case.k_self[0])
+    rc = lla.lib.lla_decode_attn_noalloc(
+        ctypes.byref(dev.cfg.c()), p(dev.packed), p(dev.rope), dev.rope.shape[0], cfg.T, case.B,
+        case.n_cap, p(dev.ctx_len), p(dev.q), p(ks), p(ks), p(dev.positions), p(dev.q_pos),
+        p(dev.c_k), p(dev.c_v), p(out), p(status),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))          # t == T: invalid
+    assert rc == lla.ERR_INVALID
+    torch.cuda.synchronize()
+    assert int(status.item()) == 12345
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
