@@ -3,14 +3,17 @@
 One step = one decode step of the workload: decode attention at each listed loop
 t over every layer's latent cache, then encode of the finished tokens (the
 per-loop K/V of the token that just completed its last loop).  Default workload:
-per-head LLA at 4x (T=4, H=16, d=128, r_k=96, r_v=160), batch 8, 4096-token
-context, one layer.
+the capacity regime, per-head LLA at 21.3x (T=4, H=16, d=128, r_k=16, r_v=32),
+batch 256, 4096-token context, all 24 shared layers back to back.
 
 Prints one JSON line (rank 0).  `value` is algorithmic HBM GB/s over the whole
-step with inputs resident in HBM; `e2e` is the same metric with the step's
-inputs copied from pinned host memory and the outputs read back inside the
-timed region.  `--impl reference` times the float64 CPU oracle on a bounded
-sample of the same workload (the reference arm of this benchmark).
+step with inputs resident in HBM; `e2e` is the same metric with each step's host
+inputs (queries, in-flight K/V, the finished tokens' per-loop rows and their new
+positions) copied in from pinned host memory and every output copied back inside
+the timed region, the latent cache resident on the device.  `sub_records` hold
+the other workloads (per-head 4x, LLA-2D, the deep-loop decode and prefill
+encode), each with its own roofline.  `--impl reference` times the float64 CPU
+oracle on a bounded sample of the same workload (the reference arm).
 """
 from __future__ import annotations
 
@@ -30,7 +33,10 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-DEFAULT_WORKLOAD = synth.WORKLOAD_ORDER[1]
+DEFAULT_WORKLOAD = "perhead_21x_T4_H16_d128_r16_32_B256_n4096_L24"
+# workloads measured as sub-records of a default run (the tiny one is a parity case)
+SUB_WORKLOADS = ("perhead_4x_T4_H16_d128_r96_160_B8_n4096", "lla2d_T4_H16_d128_r64_128_B512_n4096",
+                 "deeploop_32x_T32_H8_d96_r64_128_B16_n32768")
 METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop step"
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of the
 # current kernels (profiles/); a workload without a capture of the current code reports null.
@@ -47,13 +53,15 @@ NCU_TRAFFIC_DECOUPLED = {("perhead_4x_T4_H16_d128_r96_160_B8_n4096", 64): 276.60
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=400)
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="lla", choices=["lla", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOAD_ORDER)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-sub", action="store_true",
+                   help="measure the default workload only (no sub-records of the others)")
     p.add_argument("--encode-tokens", type=int, default=0,
                    help="override the workload's tokens encoded per step (profiling aid)")
     p.add_argument("--path", default="latent", choices=["latent", "full"],
@@ -381,49 +389,115 @@ def over_ranks(values, op, device, dist_on):
     return [float(v) for v in t]
 
 
-def cpu_baseline_sample(w, seconds: float, loops=None, d_rope=0):
-    """Time the float64 oracle on (b, h) pairs of the workload at full context."""
+def _oracle_cores():
+    """Host cores this process may run on (its CPU affinity set)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _blas_limit(n):
+    """Context manager capping the BLAS threads of NumPy at n (no-op without threadpoolctl)."""
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=int(n))
+    except Exception:  # pragma: no cover
+        import contextlib
+        return contextlib.nullcontext()
+
+
+_ORACLE_INPUTS = {}
+
+
+def _oracle_inputs(w):
+    """The oracle's codec and one sequence of workload w (drawn once per process)."""
     import torch
     import oracle as O
 
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # pragma: no cover
-        threads = 1
-    cfg = O.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
-    cod = synth.workload_codec(w)
-    codec = O.Codec(*(cod[k].astype(np.float64) for k in
-                      ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
-    x = synth.workload_tensors(w, "cpu", seed_offset=99, B=1)
-    arr = {k: (v.float().numpy().astype(np.float64) if v.dtype in (torch.bfloat16, torch.float32)
-               else v.numpy()) for k, v in x.items()}
+    if w.name not in _ORACLE_INPUTS:
+        cfg = O.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
+        cod = synth.workload_codec(w)
+        codec = O.Codec(*(cod[k].astype(np.float64) for k in
+                          ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
+        x = synth.workload_tensors(w, "cpu", seed_offset=99, B=1)
+        arr = {k: (v.float().numpy().astype(np.float64)
+                   if v.dtype in (torch.bfloat16, torch.float32) else v.numpy())
+               for k, v in x.items()}
+        _ORACLE_INPUTS[w.name] = (cfg, codec, arr)
+    return _ORACLE_INPUTS[w.name]
+
+
+def _oracle_pairs(w, seconds, loops, d_rope, threads):
+    """(b, h) pairs of workload w the float64 oracle decodes in about `seconds`,
+    with its BLAS threads capped at `threads`; returns (pairs, elapsed seconds)."""
+    import oracle as O
+
+    cfg, codec, arr = _oracle_inputs(w)
     loops = loops or w.loops
     pairs = 0
-    t0 = time.perf_counter()
-    while True:
-        h = pairs % w.H
-        t = loops[pairs % len(loops)]
-        if d_rope:
-            O.decode_attn_cache_decoupled(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"],
-                                          arr["c_k"], arr["c_v"], arr["positions"], arr["q_pos"],
-                                          arr["ctx_len"], d_rope, pairs=[(0, h)])
-        else:
-            O.decode_attn_cache(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"], arr["c_k"],
-                                arr["c_v"], arr["positions"], arr["q_pos"], arr["ctx_len"],
-                                pairs=[(0, h)])
-        pairs += 1
-        el = time.perf_counter() - t0
-        if el >= seconds and pairs >= 2:
-            break
+    with _blas_limit(threads):
+        t0 = time.perf_counter()
+        while True:
+            h = pairs % w.H
+            t = loops[pairs % len(loops)]
+            if d_rope:
+                O.decode_attn_cache_decoupled(cfg, codec, t, arr["q"], arr["k_self"],
+                                              arr["v_self"], arr["c_k"], arr["c_v"],
+                                              arr["positions"], arr["q_pos"], arr["ctx_len"],
+                                              d_rope, pairs=[(0, h)])
+            else:
+                O.decode_attn_cache(cfg, codec, t, arr["q"], arr["k_self"], arr["v_self"],
+                                    arr["c_k"], arr["c_v"], arr["positions"], arr["q_pos"],
+                                    arr["ctx_len"], pairs=[(0, h)])
+            pairs += 1
+            el = time.perf_counter() - t0
+            if el >= seconds and pairs >= 2:
+                return pairs, el
+
+
+def cpu_baseline_sample(w, seconds: float, loops=None, d_rope=0, one_thread=True):
+    """Time the float64 oracle on (b, h) pairs of the workload at full context.
+
+    The oracle runs with its BLAS threads set to the host cores this process may
+    use (``cores``); a second, shorter sample with one thread is reported beside
+    it.  GB/s are the GPU path's algorithmic bytes per (b, h) pair over the time.
+    """
+    cores = _oracle_cores()
+    share = 0.75 if one_thread else 1.0
+    pairs, el = _oracle_pairs(w, seconds * share, loops, d_rope, cores)
     per_pair = decode_bytes(w, w.n) / (w.B * w.H)
-    return {"value": pairs * per_pair / el / 1e9, "unit": "GB/s", "cores": int(threads),
-            "kind": "oracle", "seconds": round(el, 2),
-            "sample": f"{pairs} (b,h) pairs x {w.n} context tokens, loops {list(loops)}, "
-                      f"float64 NumPy; bytes scaled as the GPU path's algorithmic bytes per pair"}
+    out = {"value": pairs * per_pair / el / 1e9, "unit": "GB/s", "cores": int(cores),
+           "kind": "oracle", "seconds": round(el, 2),
+           "sample": f"{pairs} (b,h) pairs x {w.n} context tokens, loops {list(loops or w.loops)}, "
+                     f"float64 NumPy with BLAS threads = {cores} (the process's CPU affinity "
+                     f"set); bytes scaled as the GPU path's algorithmic bytes per pair"}
+    if one_thread:
+        p1, e1 = _oracle_pairs(w, seconds * (1.0 - share), loops, d_rope, 1)
+        out["value_1thread"] = p1 * per_pair / e1 / 1e9
+        out["sample_1thread"] = f"{p1} (b,h) pairs, BLAS threads = 1"
+    return out
 
 
-def run_gpu(args):
+def tflops_peak():
+    """Measured dense bf16 tensor throughput (TFLOP/s): the sustained figure, for a
+    kernel timed inside a long step, and the source of the number."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        if "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured sustained cuBLAS bf16"
+        return float(d["bf16_tflops"]), "measured burst cuBLAS bf16"
+    return 1400.0, "fallback sustained bf16"
+
+
+def decode_flops(w, n_ctx: int) -> int:
+    """Algorithmic FLOPs of one decode call: the loop-t K rebuild (2 r_k d per
+    token-head, unavoidable under full RoPE) and the latent V sum (2 r_v)."""
+    return w.B * n_ctx * w.H * 2 * (w.r_k * w.d + w.r_v)
+
+
+def init_dist():
     import torch
     import torch.distributed as dist
 
@@ -435,19 +509,22 @@ def run_gpu(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    import looped_transformer_decode_b200 as lla
+    return world, rank, local, dist_on
 
-    w = synth.WORKLOADS[args.workload]
-    if args.encode_tokens:
-        w = dataclasses.replace(w, encode_tokens=args.encode_tokens)
-    st = build_state(w, device, args.d_rope)
+
+def measure(lla, w, args, device, world, rank, local, dist_on, steps, warmup, path="latent",
+            d_rope=0, evict_arg="", eager=False, with_e2e=False):
+    """Time `steps` steps of workload w (after `warmup`), max over ranks.  Returns the
+    record of the workload (the JSON line's fields apart from the run metadata)."""
+    import torch
+
+    st = build_state(w, device, d_rope)
     n_ctx = w.n
     evict = None
-    if args.evict:
-        evict = tuple(int(v) for v in args.evict.split(","))
+    if evict_arg:
+        evict = tuple(int(v) for v in evict_arg.split(","))
         n_ctx = apply_eviction(lla, w, st, *evict)
-    full = args.path == "full"
+    full = path == "full"
     rebuild_once_ms = None
     if full:
         if evict:
@@ -461,7 +538,7 @@ def run_gpu(args):
         st["flush"] = torch.zeros(96 * 2**20, dtype=torch.int32, device=device)   # 384 MB
         l2_note = ("L2 flushed each step by a 384 MB write (inside the step time; the "
                    "decode call times exclude it)")
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         run_step(lla, w, st)
     barrier_sync(dist_on)
     # the clock sampler starts before more warm-up steps, so its first samples
@@ -477,13 +554,13 @@ def run_gpu(args):
             break
 
     ev_pairs = ([], [], [], [])
-    graphs = None if args.eager else capture_step_graphs(lla, w, st)
+    graphs = None if eager else capture_step_graphs(lla, w, st)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier_sync(dist_on)
     if clocks:
         clocks.mark_start()
     start.record()
-    for _ in range(args.steps):
+    for _ in range(steps):
         if graphs:
             replay_step_graphs(st, graphs, ev_pairs, len(w.loops) * w.layers, w.layers)
         else:
@@ -512,26 +589,52 @@ def run_gpu(args):
     if full:
         append_bytes += len(w.loops) * full_rebuild_bytes(w, st["slot"].numel())
     per_step_bytes = (len(w.loops) * w.layers * dec_bytes(w, n_ctx) + w.layers * append_bytes)
-    ms_step = ms / args.steps
+    ms_step = ms / steps
     value = world * per_step_bytes / (ms_step * 1e-3) / 1e9
     ctx_tokens = world * len(w.loops) * w.layers * w.B * n_ctx / (ms_step * 1e-3)
     peak, peak_kind = peaks()
-    # the roofline is reported for the kernel that takes most of the step: decode
-    # (prep + partial + combine per call) or, for prefill-sized encodes, the encode
-    dec_total = len(w.loops) * w.layers * dec_avg
-    enc_total = w.layers * enc_avg
-    if enc_total > dec_total:
-        unit_bytes, unit_ms = append_bytes, enc_avg
-        kname = "lla_encode + lla_full_rebuild" if full else "lla_encode"
+    dec_call = dec_bytes(w, n_ctx)
+    dec_gbs = dec_call / (dec_avg * 1e-3) / 1e9
+    enc_gbs = append_bytes / (enc_avg * 1e-3) / 1e9
+    traffic_table = NCU_TRAFFIC_FULL if full else NCU_TRAFFIC
+    traffic = ((NCU_TRAFFIC_DECOUPLED.get((w.name, d_rope)) if d_rope else traffic_table.get(w.name))
+               if not (args.encode_tokens or evict_arg) else None)
+    dkname = ("lla_full_decode_attn (full_decode_kernel [+ combine])" if full
+              else "lla_decode_attn (prep + partial kernel [+ combine])")
+    dec_roof = {"bound": "hbm", "kernel": dkname, "achieved": round(dec_gbs, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(dec_gbs / peak, 4),
+                "traffic": traffic if len(w.loops) * w.layers * dec_avg >= w.layers * enc_avg else None,
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "call_us": round(dec_avg * 1e3, 2), "algorithmic_bytes_per_call": dec_call}
+    enc_roof = {"bound": "hbm", "kernel": "lla_encode + lla_full_rebuild" if full else "lla_encode",
+                "achieved": round(enc_gbs, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(enc_gbs / peak, 4),
+                "traffic": traffic if len(w.loops) * w.layers * dec_avg < w.layers * enc_avg else None,
+                "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "call_us": round(enc_avg * 1e3, 2), "algorithmic_bytes_per_call": append_bytes,
+                "tokens_per_call": w.encode_tokens}
+    # the roofline of the kernel that takes most of the step: decode (prep + partial
+    # [+ combine] per call) or, for prefill-sized encodes, the encode
+    if len(w.loops) * w.layers * dec_avg >= w.layers * enc_avg:
+        roof = dict(dec_roof)
     else:
-        unit_bytes, unit_ms = dec_bytes(w, n_ctx), dec_avg
-        kname = ("lla_full_decode_attn (full_decode_kernel [+ combine])" if full
-                 else "lla_decode_attn (prep + partial kernel [+ combine])")
-    achieved = unit_bytes / (unit_ms * 1e-3) / 1e9
-
-    e2e = None
-    if not args.no_e2e and not full:
-        e2e = run_e2e(lla, w, st, args, dist_on, world, n_ctx)
+        roof = dict(enc_roof)
+    roof["decode_call_us"] = round(dec_avg * 1e3, 2)
+    roof["encode_call_us"] = round(enc_avg * 1e3, 2)
+    if w.mode == synth.MODE_2D and not full:
+        # LLA-2D: sixteen heads share each latent row, so the K rebuild is the tensor
+        # pipe's work (about 680 FLOP per latent byte): its bound is the tensor pipe
+        tp, tp_kind = tflops_peak()
+        fl = decode_flops(w, n_ctx)
+        tf = fl / (dec_avg * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dkname, "achieved": round(tf, 2), "peak": tp,
+                "unit": "TFLOP/s", "frac": round(tf / tp, 4), "traffic": traffic,
+                "peak_source": f"{tp_kind} (MEASURED_PEAKS.json)",
+                "algorithmic_flops_per_call": fl, "call_us": round(dec_avg * 1e3, 2),
+                "hbm": {k: dec_roof[k] for k in ("achieved", "peak", "unit", "frac",
+                                                 "algorithmic_bytes_per_call")},
+                "decode_call_us": round(dec_avg * 1e3, 2),
+                "encode_call_us": round(enc_avg * 1e3, 2)}
 
     if full:
         launches_per_step = (len(w.loops) * w.layers
@@ -540,44 +643,93 @@ def run_gpu(args):
     else:
         launches_per_step = (len(w.loops) * w.layers
                              * lla.decode_launches(st["cfg"], w.B, st["n_cap"]) + w.layers)
-    traffic_table = NCU_TRAFFIC_FULL if full else NCU_TRAFFIC
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; latents drawn in latent space as rank-R plus noise)",
-        "config": {"workload": w.name, "T": w.T, "H": w.H, "d_head": w.d, "r_k": w.r_k,
-                   "r_v": w.r_v, "mode": "per_head" if w.mode == synth.MODE_PER_HEAD else "lla_2d",
-                   "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
-                   "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
-                   "evict": list(evict) if evict else None, "attended_context": n_ctx,
-                   "path": args.path, "d_rope": args.d_rope or None,
-                   "schedule": "eager launches" if args.eager else "cuda graphs per step",
-                   "l2": l2_note},
+    rec = {
+        "value": round(value, 2), "unit": "GB/s", "steps": steps, "warmup": max(warmup, 3),
+        "ms_per_step": round(ms_step, 5),
+        "config": workload_config(w, world, evict, n_ctx, path, d_rope, eager, l2_note),
         "ctx_tokens_per_s": round(ctx_tokens, 1),
         "decode_steps_per_s": round(world * 1e3 / ms_step, 2),
-        "roofline": {"bound": "hbm", "kernel": kname,
-                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4),
-                     "traffic": ((NCU_TRAFFIC_DECOUPLED.get((w.name, args.d_rope))
-                                  if args.d_rope else traffic_table.get(w.name))
-                                 if not (args.encode_tokens or args.evict) else None),
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                     "call_us": round(unit_ms * 1e3, 2),
-                     "algorithmic_bytes_per_call": unit_bytes,
-                     "decode_call_us": round(dec_avg * 1e3, 2),
-                     "encode_call_us": round(enc_avg * 1e3, 2)},
-        "gpu_launches": launches_per_step * args.steps,
-        "e2e": e2e,
+        "roofline": roof,
+        "decode_roofline": dec_roof,
+        "encode_roofline": enc_roof,
+        "gpu_launches": launches_per_step * steps,
         "clocks": clk,
     }
     if full:
-        line["config"]["full_cache_gib"] = round(
+        rec["config"]["full_cache_gib"] = round(
             w.layers * len(w.loops) * 2 * lla.full_kv_bytes(st["cfg"], w.B, st["n_cap"]) / 2**30, 2)
-        line["config"]["rebuild_once_ms_per_layer_loop"] = round(rebuild_once_ms, 3)
-        line["e2e_note"] = "end-to-end line measured on the latent path (the default)"
+        rec["config"]["rebuild_once_ms_per_layer_loop"] = round(rebuild_once_ms, 3)
+    if with_e2e and not full:
+        if graphs:
+            del graphs
+        rec["e2e"] = run_e2e(lla, w, st, args, dist_on, world, n_ctx)
+    del st
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+def workload_config(w, world, evict=None, n_ctx=None, path="latent", d_rope=0, eager=False,
+                    l2_note=None):
+    """The JSON line's `config`: the workload by name and sizes, and how it ran."""
+    return {"workload": w.name, "T": w.T, "H": w.H, "d_head": w.d, "r_k": w.r_k,
+            "r_v": w.r_v, "mode": "per_head" if w.mode == synth.MODE_PER_HEAD else "lla_2d",
+            "batch": w.B, "context": w.n, "layers": w.layers, "loops": list(w.loops),
+            "encode_tokens": w.encode_tokens, "parallelism": f"replicas x{world}",
+            "evict": list(evict) if evict else None,
+            "attended_context": w.n if n_ctx is None else n_ctx,
+            "path": path, "d_rope": d_rope or None,
+            "schedule": "eager launches" if eager else "cuda graphs per step",
+            "l2": l2_note or (f"inputs larger than L2 ({decode_bytes(w, w.n) * w.layers / 1e6:.0f}"
+                              f" MB of latents per loop pass)")}
+
+
+def sub_record_steps(w):
+    """Timed steps of a sub-record: about two seconds of GPU time, 5 to 200 steps
+    (per-step time from the byte count at roughly half the copy bandwidth)."""
+    peak, _ = peaks()
+    est = (len(w.loops) * w.layers * decode_bytes(w, w.n) + w.layers * encode_bytes(
+        w, w.encode_tokens)) / (0.5 * peak * 1e9)
+    return int(min(200, max(5, 2.0 / max(est, 1e-6))))
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local, dist_on = init_dist()
+    device = torch.device("cuda", local)
+    import looped_transformer_decode_b200 as lla
+
+    w = synth.WORKLOADS[args.workload]
+    if args.encode_tokens:
+        w = dataclasses.replace(w, encode_tokens=args.encode_tokens)
+    rec = measure(lla, w, args, device, world, rank, local, dist_on, args.steps, args.warmup,
+                  path=args.path, d_rope=args.d_rope, evict_arg=args.evict, eager=args.eager,
+                  with_e2e=not args.no_e2e)
+    line = {"metric": METRIC, "value": rec["value"], "unit": "GB/s", "n_gpus": world,
+            "steps": rec["steps"], "warmup": rec["warmup"], "ms_per_step": rec["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; latents drawn in latent space as rank-R plus noise)",
+            "config": rec["config"], "ctx_tokens_per_s": rec["ctx_tokens_per_s"],
+            "decode_steps_per_s": rec["decode_steps_per_s"], "roofline": rec["roofline"],
+            "decode_roofline": rec["decode_roofline"], "encode_roofline": rec["encode_roofline"],
+            "gpu_launches": rec["gpu_launches"], "e2e": rec.get("e2e"), "clocks": rec["clocks"]}
+    if args.path == "full":
+        line["e2e_note"] = "no end-to-end line on the full-memory path"
+    if not args.no_sub and args.workload == DEFAULT_WORKLOAD and args.path == "latent" \
+            and not (args.d_rope or args.evict or args.encode_tokens):
+        subs = []
+        for name in SUB_WORKLOADS:
+            sw = synth.WORKLOADS[name]
+            r = measure(lla, sw, args, device, world, rank, local, dist_on, sub_record_steps(sw),
+                        3, eager=args.eager)
+            subs.append({"workload": name, **{k: r[k] for k in (
+                "value", "unit", "steps", "ms_per_step", "ctx_tokens_per_s", "decode_steps_per_s",
+                "roofline", "decode_roofline", "encode_roofline", "gpu_launches", "clocks")}})
+        line["sub_records"] = subs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = (cpu_baseline_full(w, args.cpu_seconds) if full
+        line["cpu_baseline"] = (cpu_baseline_full(w, args.cpu_seconds) if args.path == "full"
                                 else cpu_baseline_sample(w, args.cpu_seconds,
                                                          d_rope=args.d_rope))
     if rank == 0:
@@ -592,58 +744,72 @@ def cpu_baseline_full(w, seconds: float):
     (bf16-valued K/V rows drawn at random: the cost does not depend on the values)."""
     import oracle as O
 
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # pragma: no cover
-        threads = 1
+    cores = _oracle_cores()
     g = synth.rng(w.seed + 7)
     K = O.bf16_round(g.standard_normal((w.n, w.d)))
     V = O.bf16_round(g.standard_normal((w.n, w.d)))
     q, ks, vs = (g.standard_normal(w.d) for _ in range(3))
     pairs = 0
-    t0 = time.perf_counter()
-    while True:
-        O.decode_attention_full(q, ks, vs, K, V, w.n, 10000.0)
-        pairs += 1
-        el = time.perf_counter() - t0
-        if el >= seconds and pairs >= 2:
-            break
+    with _blas_limit(cores):
+        t0 = time.perf_counter()
+        while True:
+            O.decode_attention_full(q, ks, vs, K, V, w.n, 10000.0)
+            pairs += 1
+            el = time.perf_counter() - t0
+            if el >= seconds and pairs >= 2:
+                break
     per_pair = full_decode_bytes(w, w.n) / (w.B * w.H)
-    return {"value": pairs * per_pair / el / 1e9, "unit": "GB/s", "cores": int(threads),
+    return {"value": pairs * per_pair / el / 1e9, "unit": "GB/s", "cores": int(cores),
             "kind": "oracle", "seconds": round(el, 2),
             "sample": f"{pairs} (b,h) pairs x {w.n} context tokens, float64 NumPy "
                       f"decode_attention_full; bytes scaled as the GPU path's per pair"}
 
 
 def run_e2e(lla, w, st, args, dist_on, world, n_ctx):
-    """Same step with inputs copied from pinned host memory and the output read back."""
+    """The step end to end through the library's calls, with the latent cache
+    resident on the device: every decode call's query and in-flight K/V (per layer
+    and loop) and the finished tokens' per-loop rows, slots and new positions are
+    copied in from pinned host memory, and every decode output is copied back,
+    inside the timed region (eager launches; copies on the compute stream)."""
     import torch
 
-    host = []
-    h2d = 0
-    for L in st["layers"]:
-        hl = {k: L[k].cpu().pin_memory() for k in ("c_k", "c_v", "q", "k_self", "v_self",
-                                                    "positions", "q_pos", "ctx_len")}
-        host.append(hl)
-        h2d += sum(v.numel() * v.element_size() for v in hl.values())
-    hx = {"xk": st["xk"].cpu().pin_memory(), "xv": st["xv"].cpu().pin_memory()}
-    h2d += sum(v.numel() * v.element_size() for v in hx.values())
-    out_host = torch.empty(st["out"].shape, dtype=torch.float32).pin_memory()
-    d2h = out_host.numel() * 4 * len(w.loops) * w.layers
+    dev = st["out"].device
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 31)
+    shape = (w.B, w.H, w.d)
+    n_dec = len(w.loops) * w.layers
+    # per (loop, layer): q, k_self, v_self drawn once, pinned
+    hq = [[(torch.randn(shape, generator=g) / float(np.sqrt(w.d))).pin_memory(),
+           (0.2 * torch.randn(shape, generator=g)).pin_memory(),
+           (0.2 * torch.randn(shape, generator=g)).pin_memory()] for _ in range(n_dec)]
+    hx = {"xk": st["xk"].cpu().pin_memory(), "xv": st["xv"].cpu().pin_memory(),
+          "slot": st["slot"].cpu().pin_memory()}
+    hpos = {"q_pos": st["layers"][0]["q_pos"].cpu().pin_memory(),
+            "ctx_len": st["layers"][0]["ctx_len"].cpu().pin_memory()}
+    outs = [torch.empty(shape, dtype=torch.float32).pin_memory() for _ in range(n_dec)]
+    dq = [torch.empty(shape, dtype=torch.float32, device=dev) for _ in range(3)]
+    h2d = (sum(t.numel() * t.element_size() for trip in hq for t in trip)
+           + sum(v.numel() * v.element_size() for v in hx.values())
+           + w.layers * sum(v.numel() * v.element_size() for v in hpos.values()))
+    d2h = sum(o.numel() * o.element_size() for o in outs)
 
     def step():
-        for L, hl in zip(st["layers"], host):
-            for k, v in hl.items():
-                L[k].copy_(v, non_blocking=True)
-        st["xk"].copy_(hx["xk"], non_blocking=True)
-        st["xv"].copy_(hx["xv"], non_blocking=True)
+        for L in st["layers"]:                      # the new positions of this step
+            L["q_pos"].copy_(hpos["q_pos"], non_blocking=True)
+            L["ctx_len"].copy_(hpos["ctx_len"], non_blocking=True)
+        i = 0
         for t in w.loops:
             for L in st["layers"]:
-                lla.decode_attn(st["cfg"], L["packed"], st["rope"], t, L["ctx_len"], L["q"],
-                                L["k_self"], L["v_self"], L["positions"], L["q_pos"], L["c_k"],
-                                L["c_v"], out=st["out"], ws=st["ws"])
-                out_host.copy_(st["out"], non_blocking=True)
+                for dst, src in zip(dq, hq[i]):
+                    dst.copy_(src, non_blocking=True)
+                lla.decode_attn(st["cfg"], L["packed"], st["rope"], t, L["ctx_len"], dq[0], dq[1],
+                                dq[2], L["positions"], L["q_pos"], L["c_k"], L["c_v"],
+                                out=st["out"], ws=st["ws"])
+                outs[i].copy_(st["out"], non_blocking=True)
+                i += 1
+        st["xk"].copy_(hx["xk"], non_blocking=True)
+        st["xv"].copy_(hx["xv"], non_blocking=True)
+        st["slot"].copy_(hx["slot"], non_blocking=True)
         for L in st["layers"]:
             lla.encode(st["cfg"], L["packed"], st["xk"], st["xv"], st["slot"], L["c_k"], L["c_v"])
         torch.cuda.current_stream().synchronize()
@@ -659,12 +825,15 @@ def run_e2e(lla, w, st, args, dist_on, world, n_ctx):
     e.record()
     barrier_sync(dist_on)
     ms = s.elapsed_time(e) / steps
-    ms = over_ranks([ms], "max", st["out"].device, dist_on)[0]
+    ms = over_ranks([ms], "max", dev, dist_on)[0]
     per_step_bytes = (len(w.loops) * w.layers * decode_bytes(w, n_ctx)
                       + w.layers * encode_bytes(w, w.encode_tokens))
     return {"value": round(world * per_step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "steps": steps}
+            "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "inputs": "per decode call: q, k_self, v_self; per step: the finished tokens' "
+                      "per-loop K/V rows, their cache slots, q_pos and ctx_len; outputs: every "
+                      "decode call's [B, H, d]; latent cache resident in HBM"}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -675,14 +844,16 @@ def run_reference(args):
     if rank != 0:
         return
     w = synth.WORKLOADS[args.workload]
-    per_step = max(1.0, args.cpu_seconds / 4)
+    # each step a bounded sample, so that the whole run stays near two minutes
+    per_step = min(max(0.05, args.cpu_seconds / 4), 120.0 / max(1, args.steps))
     vals = []
+    _oracle_inputs(w)                 # the inputs are drawn once, outside the timed steps
     for _ in range(args.warmup):
-        cpu_baseline_sample(w, per_step / 4)
+        cpu_baseline_sample(w, per_step / 4, one_thread=False)
     t0 = time.perf_counter()
     last = None
     for _ in range(args.steps):
-        last = cpu_baseline_sample(w, per_step)
+        last = cpu_baseline_sample(w, per_step, one_thread=False)
         vals.append(last["value"])
     el = time.perf_counter() - t0
     value = float(np.mean(vals))
@@ -691,9 +862,7 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el * 1e3 / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "H": w.H, "d_head": w.d, "r_k": w.r_k,
-                   "r_v": w.r_v, "batch": w.B, "context": w.n, "layers": w.layers,
-                   "loops": list(w.loops), "parallelism": "host cores, rank 0 only"},
+        "config": workload_config(w, world),
         "cpu_baseline": {"kind": "oracle", "cores": last["cores"], "value": round(value, 4),
                          "unit": "GB/s", "sample": last["sample"] + f"; {per_step:.1f} s per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,

@@ -85,6 +85,12 @@ struct TcParams {
   uint32_t comb_off;                         // smem: olat [r_v], split weights [64], reductions
   int fuse_combine;                          // 1: the combine is done here (one split per group)
   uint32_t p_buf_bytes;
+  // phase-operand kernel (decode_tcf_kernel): ne buffers of the phase operand E
+  // ([128 tokens x d] bf16 each), F columns n_f = G r_k + 16, bytes of one item's
+  // operand image, and the swizzle mask of the K latent tile (7: 128-byte rows,
+  // 3: 64-byte rows)
+  uint32_t e_off, e_bytes, b_img_bytes;
+  int ne, n_f, kswz_mask;
   const float2* rope;    // [rope_max_pos][d/2]
   const int32_t* ctx_len;
   const int32_t* positions;
@@ -435,6 +441,16 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
   }
 }
 
+// Before the CTA frees TMEM: arrive on `bar` once every MMA this thread issued has
+// completed, and wait for that (bounded).  In a normal run they all have completed
+// already (the epilogue waited on their commits); after an abort some may not have.
+__device__ __forceinline__ void mma_drain(uint64_t* bar) {
+  mma_commit(bar);
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, 0) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+  }
+}
+
 // log2 of the largest softmax weight a tile may carry before the V accumulator
 // is rescaled to a new reference maximum.
 constexpr float kRescaleLog2 = 8.f;
@@ -534,6 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bempty = bfull + 2;          // [2] operand buffer free
   uint64_t* pfull = bempty + 2;          // [2] softmax weights written
   uint64_t* pempty = pfull + 2;          // [2] V MMA done with the weights buffer
+  uint64_t* drain = pempty + 2;          // [2] each MMA issuer's last MMAs completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
 
@@ -558,6 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pfull[a], 4);
       mbar_init(&pempty[a], 1);
     }
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -725,6 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (k == r.ntiles - 1) mma_commit(&bempty[buf]);   // last use of this B buffer
         }
       }
+      mma_drain(&drain[0]);
     }
     __syncwarp();
   } else if (warp == kVMmaWarp) {
@@ -766,6 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&empty_v[vs]);
         }
       }
+      mma_drain(&drain[1]);
     }
     __syncwarp();
   } else {
@@ -1159,6 +1180,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
   uint64_t* bempty = bfull + 2;          // [nbuf_b] operand buffer free
   uint64_t* pfull = bempty + 2;          // [2] softmax weights written
   uint64_t* pempty = pfull + 2;          // [2] V MMA done with the weights buffer
+  uint64_t* drain = pempty + 2;          // [2] each MMA issuer's last MMAs completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
 
@@ -1185,6 +1207,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
       mbar_init(&pfull[a], 4 * HP);
       mbar_init(&pempty[a], 1);
     }
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1340,6 +1364,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           if (k == r.ntiles - 1) mma_commit(&bempty[buf]);   // last use of this B buffer
         }
       }
+      mma_drain(&drain[0]);
     }
     __syncwarp();
   } else if (warp == kVMmaWarp2) {
@@ -1381,6 +1406,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           mma_commit(&empty_v[vs]);
         }
       }
+      mma_drain(&drain[1]);
     }
     __syncwarp();
   } else {
@@ -1598,6 +1624,690 @@ __global__ void __launch_bounds__(kThreads2, 1)
   }
 }
 
+// ------------------------------------------------------------------ phase-operand kernel
+//
+// Per head, small latent ranks.  The score of history token j is (decode_prep_kernel's
+// reordering)
+//   s_j = Re sum_i U_{j,i} e^{i p_j theta_i},   U_j = c_j A~ + M~,
+// with A~ = kappa conj(q~) W~ the query-absorbed up-projection and M~ its bias.
+// With E_j = (cos p_j theta_i, -sin p_j theta_i)_i (two entries per RoPE pair) and
+// B_m = (Re A~_{m,i}, Im A~_{m,i})_i for latent index m,
+//   s_j = sum_m c_{j,m} F_{j,m} + F_{j,M},   F = E B^T,
+// where F_{j,M} is the same product for the bias row M~.  E depends only on the
+// tokens' positions, so one MMA per 128-token tile (M = 128, K = d, N = G r_k + 16:
+// the G heads' rows B_m plus their bias rows as bf16 hi + lo) gives F for every head
+// of the item, and the epilogue finishes each token-head with r_k FMAs against its
+// latents instead of d/2 complex products.  The V sum is taken transposed for the G
+// heads at once, D_v^T[G r_v x 2G] += C_v^T P^T, of which only the diagonal blocks
+// are read (as in the LLA-2D kernel).  Both are exact reorderings of the same sums.
+
+// Operand image of one item (sequence b, group of G heads) for decode_tcf_kernel:
+// [n_f rows x d] bf16 in the 128-byte-swizzled K-major layout (d / 64 column blocks
+// of n_f x 128 bytes; 16-byte chunk c of row n at chunk c ^ (n % 8)).  Row g r_k + m
+// is B_m of head g, rows G r_k + 2g and + 1 its bias M~ as bf16 hi and lo, the rest
+// zero.  One CTA of 128 threads per (h, b).
+template <int D>
+__global__ void __launch_bounds__(128) decode_prep_f_kernel(
+    const float* __restrict__ q, const int32_t* __restrict__ q_pos, const float2* __restrict__ rope,
+    int rope_max_pos, const float* __restrict__ wupk_t, const float* __restrict__ muk_t, float kappa,
+    int H, int r_k, int G, int n_f, uint32_t img_bytes, unsigned char* __restrict__ ops,
+    int32_t* status, uint32_t* counters) {
+  constexpr int HALF = D / 2;
+  constexpr int EBLK = D / 64;
+  // the partial kernel may start its prologue and latent loads now; it waits for
+  // this grid before it reads the images or the counter
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float2 qc[HALF];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int g = h % G;
+  if (counters && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0)
+    counters[(size_t)gridDim.y * H] = 0u;
+  int qp = q_pos[b];
+  if (qp < 0 || qp >= rope_max_pos) {
+    if (tid == 0 && h == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
+    qp = 0;
+  }
+  const float* qh = q + ((size_t)b * H + h) * D;
+  for (int i = tid; i < HALF; i += 128) {
+    const float2 e = rope[(size_t)qp * HALF + i];
+    const float x0 = qh[i], x1 = qh[i + HALF];
+    qc[i] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
+  }
+  __syncthreads();
+  const float* W = wupk_t + (size_t)h * D * r_k;   // [d][r_k]
+  const float* mu = muk_t + (size_t)h * D;
+  unsigned char* img = ops + ((size_t)b * (H / G) + h / G) * img_bytes;
+  // this head's rows: its r_k rows, its two bias rows, and (first head of the group)
+  // the zero rows that pad n_f
+  const int pad0 = G * r_k + 2 * G;
+  const int rows = r_k + 2 + (g == 0 ? n_f - pad0 : 0);
+  for (int idx = tid; idx < rows * EBLK * 8; idx += 128) {
+    const int lr = idx / (EBLK * 8), kb = (idx >> 3) % EBLK, c = idx & 7;
+    const int n = lr < r_k ? g * r_k + lr
+                           : (lr < r_k + 2 ? G * r_k + 2 * g + (lr - r_k) : pad0 + (lr - r_k - 2));
+    __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = kb * 32 + c * 4 + e;       // RoPE pair of entries 2e, 2e + 1
+      const float2 z = qc[i];
+      float re = 0.f, im = 0.f;
+      if (lr < r_k) {
+        const float wr = W[(size_t)i * r_k + lr], wi = W[(size_t)(i + HALF) * r_k + lr];
+        re = kappa * (z.x * wr + z.y * wi);
+        im = kappa * (z.x * wi - z.y * wr);
+      } else if (lr < r_k + 2) {
+        const float mr = mu[i], mi = mu[i + HALF];
+        re = kappa * (z.x * mr + z.y * mi);
+        im = kappa * (z.x * mi - z.y * mr);
+        if (lr == r_k + 1) {   // lo row: what the bf16 hi row leaves
+          re -= __bfloat162float(__float2bfloat16_rn(re));
+          im -= __bfloat162float(__float2bfloat16_rn(im));
+        }
+      }
+      v[2 * e] = __float2bfloat16_rn(re);
+      v[2 * e + 1] = __float2bfloat16_rn(im);
+    }
+    *reinterpret_cast<uint4*>(img + (size_t)kb * n_f * 128 + (size_t)n * 128 + ((c ^ (n & 7)) << 4)) =
+        *reinterpret_cast<const uint4*>(v);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v.x, v.y);   // .x in the low half
+  uint32_t u;
+  memcpy(&u, &b, 4);
+  return u;
+}
+
+// bf16 pair (low half first) -> two floats
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// D: head width; G: heads per item (G r_v = 128, the M of the V MMA); KP: r_k.
+// Warps as in decode_tc_kernel: 0 K latent producer (and each item's operand image),
+// 1 F MMA issuer, 2..9 epilogue (two warpgroups: warpgroup w owns heads
+// [w G/2, (w + 1) G/2) of the item for scores and softmax, and half of the RoPE pairs
+// of the phase tiles it writes), 10 V latent producer, 11 V MMA issuer.
+template <int D, int G, int KP, bool FUSE>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tcf_kernel(const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
+  constexpr int HW = G / kEpiWG;             // heads per epilogue warpgroup
+  constexpr int WG_PAIRS = D / 2 / kEpiWG;   // RoPE pairs of a token row each warpgroup writes
+  constexpr int NBIAS = 2 * G <= 8 ? 8 : 16; // bias columns read (hi, lo of every head)
+  static_assert(HW >= 1 && WG_PAIRS % 4 == 0 && KP % 16 == 0, "shape");
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(sm + p.bar_off);   // [nst] K latent tile landed
+  uint64_t* empty_k = full_k + p.nst;                                // [nst] epilogue read it
+  uint64_t* full_v = empty_k + p.nst;                                // [nst_v] V latent tile landed
+  uint64_t* empty_v = full_v + p.nst_v;                              // [nst_v] V MMA done with it
+  uint64_t* efull = empty_v + p.nst_v;   // [2] phase tile written
+  uint64_t* tfull = efull + 2;           // [3] F in TMEM
+  uint64_t* tempty = tfull + 3;          // [3] F read
+  uint64_t* bfull = tempty + 3;          // [2] item operand image loaded
+  uint64_t* bempty = bfull + 2;          // [2] operand buffer free
+  uint64_t* pfull = bempty + 2;          // [2] softmax weights written
+  uint64_t* pempty = pfull + 2;          // [2] V MMA done with the weights buffer
+  uint64_t* drain = pempty + 2;          // [2] each MMA issuer's last MMAs completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.nst; ++s) {
+      mbar_init(&full_k[s], 1);
+      mbar_init(&empty_k[s], kEpiWarps);
+    }
+    for (int s = 0; s < p.nst_v; ++s) {
+      mbar_init(&full_v[s], 1);
+      mbar_init(&empty_v[s], 1);
+    }
+    for (int a = 0; a < 3; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiWarps);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&efull[a], kEpiWarps);
+      mbar_init(&bfull[a], 1);
+      mbar_init(&bempty[a], 1);
+      mbar_init(&pfull[a], kEpiWarps);
+      mbar_init(&pempty[a], 1);
+    }
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp >= 2 && warp < 2 + kEpiWarps) {
+    const int et = threadIdx.x - 64;
+    if (ctx_s) {
+      int* cs = reinterpret_cast<int*>(sm + p.ctx_off);
+      for (int b = et; b < p.B; b += kEpiThreads) {
+        int n = p.ctx_len[b];
+        if (n < 0 || n > p.n_cap) {
+          if (blockIdx.x == 0) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
+          n = n < 0 ? 0 : p.n_cap;
+        }
+        cs[b] = n;
+      }
+    }
+    if (et < 64) {
+      reinterpret_cast<float2*>(sm + p.rope_off)[et] = p.step[et];
+      reinterpret_cast<uint2*>(sm + p.rope_off + 512)[et] = make_uint2(p.phi_lo[et], p.phi_hi[et]);
+    }
+    // both weight buffers start zero: rows >= 2G are never written
+    for (int idx = et; idx < 2 * 4096 / 4; idx += kEpiThreads)
+      reinterpret_cast<uint32_t*>(sm + p.p_off)[idx] = 0u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 || warp == kVProdWarp) {
+    // ------------------------------------------------------------ TMA producers
+    if (lane == 0) {
+      const bool kside = warp == 0;
+      const CUtensorMap* map = kside ? &map_k : &map_v;
+      tma_prefetch_desc(map);
+      const int nst = kside ? p.nst : p.nst_v;
+      uint64_t* fullb = kside ? full_k : full_v;
+      uint64_t* emptyb = kside ? empty_k : empty_v;
+      uint32_t it = 0, jn = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        if (r.ntiles == 0) continue;
+        if (kside) {
+          // the item's operand image (written by the prep grid, which may still be
+          // running when this kernel starts)
+          if (jn == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+          const uint32_t buf = jn % p.nbuf_b, bph = (jn / p.nbuf_b) & 1u;
+          if (!mbar_wait(&bempty[buf], bph ^ 1u, abort_flag)) break;
+          const size_t unit = (size_t)r.b * p.HG + r.hg;
+          mbar_arrive_expect_tx(&bfull[buf], p.b_img_bytes);
+          bulk_load(sm + p.b_off + buf * p.b_head_bytes, p.ops_b + unit * p.b_img_bytes,
+                    p.b_img_bytes, &bfull[buf]);
+          ++jn;
+        }
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t stage = it % nst, ph = (it / nst) & 1u;
+          if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int y = r.tok0 + k * kTile;
+          if (kside) {
+            mbar_arrive_expect_tx(&fullb[stage], p.tx_bytes);
+            unsigned char* st = sm + p.st_off + stage * p.st_bytes;
+            for (int kb = 0; kb < p.nkb; ++kb)
+              tma_load_3d(st + kb * p.box_bytes, map, &fullb[stage],
+                          r.hg * (G * KP) + kb * p.box_k, y, r.b);
+          } else {
+            mbar_arrive_expect_tx(&fullb[stage], p.tx_v);
+            unsigned char* st = sm + p.stv_off + stage * p.stv_bytes;
+            for (int vb = 0; vb < p.nvb; ++vb)
+              tma_load_3d(st + vb * p.vbox_bytes, map, &fullb[stage],
+                          r.hg * (G * p.r_v) + vb * p.cvb, y, r.b);
+          }
+        }
+      }
+      if (*abort_flag) {
+        // Drain: wait (bounded) for every copy this thread issued before leaving.
+        const uint32_t n_out = it < (uint32_t)nst ? it : (uint32_t)nst;
+        for (uint32_t j = 0; j < n_out; ++j) {
+          const uint32_t i = it - 1 - j;
+          const uint32_t stage = i % nst, ph = (i / nst) & 1u;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&fullb[stage], ph) && global_timer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+        for (uint32_t j = 0; kside && j < (uint32_t)p.nbuf_b && j < jn; ++j) {
+          const uint32_t i = jn - 1 - j;
+          const unsigned long long t0 = global_timer_ns();
+          while (!mbar_try_wait(&bfull[i % p.nbuf_b], (i / p.nbuf_b) & 1u) &&
+                 global_timer_ns() - t0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ F MMA issuer
+    // F[acc] = E (128 tokens x d, K-major) x B^T (n_f rows x d, K-major): K = d in
+    // steps of 16, each a 32-byte slice of a 128-byte-swizzled column block.
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, p.n_f);
+      const uint32_t e_base = smem_addr(sm + p.e_off);
+      const uint32_t b_base0 = smem_addr(sm + p.b_off);
+      uint32_t it = 0, jn = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        if (r.ntiles == 0) continue;
+        const uint32_t buf = jn % p.nbuf_b, bph = (jn / p.nbuf_b) & 1u;
+        if (!mbar_wait(&bfull[buf], bph, abort_flag)) break;
+        ++jn;
+        const uint32_t b_base = b_base0 + buf * p.b_head_bytes;
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t e = it % p.ne, eph = (it / p.ne) & 1u;
+          const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+          if (!mbar_wait(&efull[e], eph, abort_flag) ||
+              !mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * p.n_f;
+          const uint32_t e_addr = e_base + e * p.e_bytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t blk = kk >> 2, koff = (kk & 3) * 32;
+            const uint64_t adesc = smem_desc(e_addr + blk * (kTile * 128) + koff, 16, 1024, 2);
+            const uint64_t bdesc = smem_desc(b_base + blk * (p.n_f * 128) + koff, 16, 1024, 2);
+            mma_bf16(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&tfull[acc]);
+          if (k == r.ntiles - 1) mma_commit(&bempty[buf]);   // last use of this image
+        }
+      }
+      mma_drain(&drain[0]);
+    }
+    __syncwarp();
+  } else if (warp == kVMmaWarp) {
+    // ------------------------------------------------------------ V MMA issuer
+    // D_v^T (G r_v = 128 latent dims x 16) (+)= C_v^T (128 x 128 tokens, MN-major A,
+    // two 64-dim boxes) x P^T (128 tokens x 16 weight rows, K-major B).
+    if (lane == 0) {
+      const uint32_t idesc_v = idesc_bf16_f32(128, 16) | (1u << 15);   // A (c_v^T) MN-major
+      const uint32_t sbo_v = 16u * p.cvb;
+      const uint32_t p_base = smem_addr(sm + p.p_off);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        for (int k = 0; k < r.ntiles; ++k, ++it) {
+          const uint32_t pb = it & 1u;
+          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag) ||
+              !mbar_wait(&full_v[vs], vph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(sm + p.stv_off + vs * p.stv_bytes);
+          const uint32_t b_addr = p_base + pb * 4096u;
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t adesc = smem_desc(a_addr + kk * 2 * sbo_v, p.vbox_bytes, sbo_v, 2);
+            const uint64_t bdesc = smem_desc(b_addr + kk * 256, 128, 2048, 0);
+            mma_bf16(tmem_base + p.v_col0, adesc, bdesc, idesc_v, (k == 0 && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(&pempty[pb]);
+          mma_commit(&empty_v[vs]);
+        }
+      }
+      mma_drain(&drain[1]);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;
+    const int wgi = (warp - 2) >> 2;          // warpgroup: heads [wgi HW, (wgi + 1) HW)
+    const int sub = warp & 3;                 // TMEM sub-partition of this warp
+    const int row = sub * 32 + lane;          // token row of the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+    float* red = reinterpret_cast<float*>(sm + p.red_off);     // [G][4]
+    float* olat = reinterpret_cast<float*>(sm + p.comb_off);   // [128]: lane g r_v + m
+    float* misc = olat + 128;   // [64]: m per head [0, G), q . k_self partials [8, 8 + 4G)
+
+    // Phase tiles: the RoPE factors conj(e^{i p theta_i}) of this warpgroup's pairs at
+    // this thread's token row of the last tile written, advanced by one complex
+    // product when the next tile's token sits a tile further on (as in
+    // decode_tc_kernel), and a cursor over the tiles still to write.
+    TileCursor ec;
+    cursor_first(p, ctx_s, ec);
+    float2 ef[WG_PAIRS];
+    int pos_cur = kNoPos, run = 0;
+    const float2* step_s = reinterpret_cast<const float2*>(sm + p.rope_off) + wgi * WG_PAIRS;
+    const uint2* phi_s = reinterpret_cast<const uint2*>(sm + p.rope_off + 512) + wgi * WG_PAIRS;
+    auto advance_rope = [&](int praw) {
+      if (praw == kNoPos) return;               // row past the context: keep factors
+      const int pn = checked_pos(p, praw);
+      if (pos_cur != kNoPos && pn == pos_cur + kTile && run < kReseedTiles) {
+#pragma unroll
+        for (int q = 0; q < WG_PAIRS; ++q) {
+          const float2 st = step_s[q];
+          const float2 e = ef[q];
+          ef[q] = make_float2(fmaf(e.x, st.x, -e.y * st.y), fmaf(e.x, st.y, e.y * st.x));
+        }
+        ++run;
+      } else {
+#pragma unroll
+        for (int q = 0; q < WG_PAIRS; ++q) {
+          const uint2 ph = phi_s[q];
+          ef[q] = rope_factor(static_cast<uint32_t>(pn), ph.x, ph.y);
+        }
+        run = 0;
+      }
+      pos_cur = pn;
+    };
+#pragma unroll
+    for (int q = 0; q < WG_PAIRS; ++q) ef[q] = make_float2(1.f, 0.f);
+    uint32_t ie = 0;   // phase tiles written
+    // Write this thread's row of the next phase tile into buffer ie % ne: entries
+    // (2i, 2i + 1) = (cos, -sin) of pair i, 128-byte swizzled K-major rows.
+    auto write_e = [&]() {
+      advance_rope(cursor_pos(p, ec, row));
+      unsigned char* eb = sm + p.e_off + (ie % p.ne) * p.e_bytes;
+#pragma unroll
+      for (int c = 0; c < WG_PAIRS / 4; ++c) {
+        const int pair0 = wgi * WG_PAIRS + c * 4;
+        const int blk = pair0 >> 5, ch = (pair0 >> 2) & 7;
+        uint4 v;
+        v.x = pack_bf16x2(ef[c * 4 + 0]);
+        v.y = pack_bf16x2(ef[c * 4 + 1]);
+        v.z = pack_bf16x2(ef[c * 4 + 2]);
+        v.w = pack_bf16x2(ef[c * 4 + 3]);
+        *reinterpret_cast<uint4*>(eb + blk * (kTile * 128) + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&efull[ie % p.ne]);
+      cursor_next(p, ctx_s, ec);
+      ++ie;
+    };
+    for (int k = 0; k < p.ne && ec.valid; ++k) write_e();
+
+    uint32_t it = 0;
+    bool aborted = false;
+    for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
+      const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
+      float m_ref[HW], l_part[HW];
+#pragma unroll
+      for (int hh = 0; hh < HW; ++hh) {
+        m_ref[hh] = -INFINITY;
+        l_part[hh] = 0.f;
+      }
+      if constexpr (FUSE) {
+        // fused finish, set up while the tiles stream: the in-flight scores' partial
+        // dot products q . k_self (per warp of warpgroup 0), and the heads' W_up,v rows
+        // into L2, kept there ahead of the latent stream
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const size_t bh = (size_t)r.b * p.H + r.hg * G + g;
+          if (wgi == 0) {
+            const float qk = row < p.d ? __ldg(p.q + bh * p.d + row) * __ldg(p.k_self + bh * p.d + row) : 0.f;
+            const float sdot = warp_sum_f(qk);
+            if (lane == 0) misc[8 + g * 4 + sub] = sdot;
+          }
+          const char* wrow = reinterpret_cast<const char*>(p.wupv_t + (size_t)(r.hg * G + g) * p.d * p.r_v);
+          for (int off = et * 128; off < p.d * p.r_v * 4; off += kEpiThreads * 128)
+            asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wrow + off));
+        }
+      }
+      for (int k = 0; k < r.ntiles; ++k, ++it) {
+        const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+        const uint32_t stage = it % p.nst, kph = (it / p.nst) & 1u;
+        const int t0 = r.tok0 + k * kTile;
+        const int cnt = min(kTile, r.tok_end - t0);
+        const bool valid = row < cnt;
+
+        bool ok = mbar_wait(&tfull[acc], aph, abort_flag);
+        tc_fence_after();
+        float f[HW][KP];
+        float fb[NBIAS];
+#pragma unroll
+        for (int hh = 0; hh < HW; ++hh) {
+          const uint32_t col = tmem_base + lane_addr + acc * p.n_f + (wgi * HW + hh) * KP;
+#pragma unroll
+          for (int c = 0; c < KP / 16; ++c) tmem_ld16(col + c * 16, &f[hh][c * 16]);
+        }
+        if constexpr (NBIAS == 8)
+          tmem_ld8(tmem_base + lane_addr + acc * p.n_f + G * KP, fb);
+        else
+          tmem_ld16(tmem_base + lane_addr + acc * p.n_f + G * KP, fb);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+        // one phase buffer: the next tile's E goes in as soon as F of this one is out
+        if (p.ne == 1 && ec.valid) write_e();
+
+        // s = sum_m c_m F_m + F_M for each of this warpgroup's heads, with this token
+        // row's latents read from the swizzled K tile
+        ok = ok && mbar_wait(&full_k[stage], kph, abort_flag);
+        float s[HW];
+        {
+          const unsigned char* st = sm + p.st_off + stage * p.st_bytes;
+          const uint32_t row_bytes = (uint32_t)p.box_k * 2;
+#pragma unroll
+          for (int hh = 0; hh < HW; ++hh) {
+            const int e0 = (wgi * HW + hh) * KP;           // first latent column of the head
+            const unsigned char* bx = st + (e0 / p.box_k) * p.box_bytes;
+            const uint32_t c0 = (uint32_t)(e0 % p.box_k) * 2 / 16;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < KP / 8; ++cc) {
+              const uint32_t L = row * row_bytes + (c0 + cc) * 16;
+              const uint4 w = *reinterpret_cast<const uint4*>(
+                  bx + (L ^ (((L >> 7) & (uint32_t)p.kswz_mask) << 4)));
+              const float* fr = &f[hh][cc * 8];
+              a0 = fmaf(bf_lo(w.x), fr[0], a0);
+              a1 = fmaf(bf_hi(w.x), fr[1], a1);
+              a0 = fmaf(bf_lo(w.y), fr[2], a0);
+              a1 = fmaf(bf_hi(w.y), fr[3], a1);
+              a0 = fmaf(bf_lo(w.z), fr[4], a0);
+              a1 = fmaf(bf_hi(w.z), fr[5], a1);
+              a0 = fmaf(bf_lo(w.w), fr[6], a0);
+              a1 = fmaf(bf_hi(w.w), fr[7], a1);
+            }
+            const int g = wgi * HW + hh;
+            s[hh] = valid ? (a0 + a1) + (fb[2 * g] + fb[2 * g + 1]) : -INFINITY;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_k[stage]);
+        if (epi_barrier_or(!ok)) {
+          aborted = true;
+          break;
+        }
+        // ---- softmax weights against the item's reference maximum (taken on the
+        // item's first tile; a later tile takes a new one only when a score exceeds it
+        // by more than 2^kRescaleLog2), per head, within the owning warpgroup
+        int over = 0;
+#pragma unroll
+        for (int hh = 0; hh < HW; ++hh) over |= s[hh] > m_ref[hh] + kRescaleLog2;
+        bool rescale = false;
+        float alpha[HW];
+#pragma unroll
+        for (int hh = 0; hh < HW; ++hh) alpha[hh] = 1.f;
+        if (k == 0 || wg_barrier_or(2 + wgi, over)) {
+#pragma unroll
+          for (int hh = 0; hh < HW; ++hh) {
+            const float mx = warp_max_f(s[hh]);
+            if (lane == 0) red[(wgi * HW + hh) * 4 + sub] = mx;
+          }
+          named_barrier(2 + wgi, 128);
+#pragma unroll
+          for (int hh = 0; hh < HW; ++hh) {
+            const int g = wgi * HW + hh;
+            const float mt =
+                fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
+            if (k == 0) {
+              m_ref[hh] = mt;
+            } else if (mt > m_ref[hh] + kRescaleLog2) {
+              alpha[hh] = exp2f(m_ref[hh] - mt);
+              m_ref[hh] = mt;
+              rescale = true;
+            }
+          }
+          named_barrier(2 + wgi, 128);   // every warp has read red before it is reused
+        }
+        const uint32_t pb = it & 1u;
+        // the weights buffer is free once the V MMA of tile it - 2 has finished
+        ok = mbar_wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u, abort_flag);
+        if (rescale) {
+          // rare: rescale columns 2g, 2g + 1 of the V accumulator (every lane this
+          // warp owns) once the V MMA of the previous tile has finished
+          ok = ok && mbar_wait(&pempty[(it - 1) & 1u], ((it - 1) >> 1) & 1u, abort_flag);
+          tc_fence_after();
+#pragma unroll
+          for (int hh = 0; hh < HW; ++hh) {
+            if (alpha[hh] != 1.f) {
+              const uint32_t ta = tmem_base + lane_addr + p.v_col0 + 2 * (wgi * HW + hh);
+              float v[2];
+              tmem_ld2(ta, v);
+              tmem_wait_ld();
+              tmem_st2(ta, v[0] * alpha[hh], v[1] * alpha[hh]);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        if (cnt < kTile && wgi == 0) {
+          // rows past the context: zero them in the V stage, so that the V MMA takes
+          // zero weights times zeros whatever the cache holds there
+          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          ok = ok && mbar_wait(&full_v[vs], vph, abort_flag);
+          if (!valid) {
+            unsigned char* vrow = sm + p.stv_off + vs * p.stv_bytes + row * 128;
+            for (int vb = 0; vb < p.nvb; ++vb)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(vrow + vb * p.vbox_bytes + c * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int hh = 0; hh < HW; ++hh) {
+          const int g = wgi * HW + hh;
+          const float pj = valid ? exp2f(s[hh] - m_ref[hh]) : 0.f;
+          l_part[hh] = l_part[hh] * alpha[hh] + pj;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(pj);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(pj - __bfloat162float(hi));
+          // weight rows 2g (hi) and 2g + 1 (lo): row group (2g) / 8, rows (2g) % 8 and + 1
+          unsigned char* pg = sm + p.p_off + pb * 4096u + ((2 * g) >> 3) * 2048 +
+                              (row >> 3) * 128 + ((2 * g) & 7) * 16 + (row & 7) * 2;
+          *reinterpret_cast<__nv_bfloat16*>(pg) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(pg + 16) = lo;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pfull[pb]);   // one arrival per epilogue warp
+        if (!ok) *abort_flag = 1;
+        // two phase buffers: the tile after next goes into this tile's buffer (its
+        // last reader, this tile's F MMA, has completed)
+        if (p.ne == 2 && ec.valid) write_e();
+      }
+      if (aborted) break;
+      // ---------------------------------------------------------- item finish
+      // this warpgroup's heads: l over the item (per warp into red), m
+#pragma unroll
+      for (int hh = 0; hh < HW; ++hh) {
+        const int g = wgi * HW + hh;
+        const float l = warp_sum_f(l_part[hh]);
+        if (lane == 0) red[g * 4 + sub] = l;
+        if (row == 0) misc[g] = m_ref[hh];
+      }
+      bool okv = true;
+      if (r.ntiles > 0) {
+        const uint32_t last = it - 1;
+        okv = __all_sync(0xffffffffu, mbar_wait(&pempty[last & 1u], (last >> 1) & 1u, abort_flag));
+        tc_fence_after();
+      }
+      named_barrier(1, kEpiThreads);            // red, misc visible; olat free
+      // TMEM lane g r_v + m holds head g's latent dim m in columns 2g (hi), 2g + 1 (lo)
+      const int gl = row / p.r_v;               // head of this warp's lanes (r_v >= 32)
+      if (wgi == 0) {
+        float v[2] = {0.f, 0.f};
+        if (r.ntiles > 0 && okv) {
+          tmem_ld2(tmem_base + lane_addr + p.v_col0 + 2 * gl, v);
+          tmem_wait_ld();
+        }
+        olat[row] = v[0] + v[1];
+      }
+      tc_fence_before();
+      named_barrier(1, kEpiThreads);            // olat complete
+      if constexpr (FUSE) {
+        // One split per group: o = (W_up,v o_lat a + mu_v l a + v_self b) / (l a + b),
+        // a = 2^(m - M), b = 2^(s_self - M), M = max(m, s_self) (base-2 scores).
+        for (int o = et; o < G * p.d; o += kEpiThreads) {
+          const int g = o / p.d, dd = o - g * p.d;
+          const int h = r.hg * G + g;
+          const size_t bh = (size_t)r.b * p.H + h;
+          const float m_h = r.ntiles > 0 ? misc[g] : -INFINITY;
+          const float l_h = (red[g * 4] + red[g * 4 + 1]) + (red[g * 4 + 2] + red[g * 4 + 3]);
+          const float s_self = p.kappa * ((misc[8 + g * 4] + misc[8 + g * 4 + 1]) +
+                                          (misc[8 + g * 4 + 2] + misc[8 + g * 4 + 3]));
+          const float M = fmaxf(m_h, s_self);
+          const float a = r.ntiles > 0 ? exp2f(m_h - M) : 0.f, bsf = exp2f(s_self - M);
+          const float inv = 1.f / (l_h * a + bsf);
+          const float* Wt = p.wupv_t + (size_t)h * p.d * p.r_v + dd;
+          const float* ol = olat + g * p.r_v;
+          float y0 = 0.f, y1 = 0.f;
+          for (int m0 = 0; m0 < p.r_v; m0 += 16) {
+            float wv[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) wv[e] = __ldg(Wt + (size_t)(m0 + e) * p.d);
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              y0 = fmaf(wv[e], ol[m0 + e], y0);
+              y1 = fmaf(wv[e + 1], ol[m0 + e + 1], y1);
+            }
+          }
+          p.out[bh * p.d + dd] = ((y0 + y1) * a + __ldg(p.muv_t + (size_t)h * p.d + dd) * (l_h * a) +
+                                  __ldg(p.v_self + bh * p.d + dd) * bsf) * inv;
+        }
+      } else {
+        // split partials (m, l, sum p c_v) of the group's heads for decode_combine_kernel
+        for (int idx = et; idx < G * (2 + p.r_v); idx += kEpiThreads) {
+          const int g = idx / (2 + p.r_v), m = idx - g * (2 + p.r_v);
+          const size_t bh = (size_t)r.b * p.H + r.hg * G + g;
+          float v;
+          if (r.ntiles == 0)
+            v = m == 0 ? -INFINITY : 0.f;
+          else if (m == 0)
+            v = misc[g];
+          else if (m == 1)
+            v = (red[g * 4] + red[g * 4 + 1]) + (red[g * 4 + 2] + red[g * 4 + 3]);
+          else
+            v = olat[g * p.r_v + m - 2];
+          p.partials[(bh * p.S + r.s) * (2 + p.r_v) + m] = v;
+        }
+      }
+      named_barrier(1, kEpiThreads);            // scratch free for the next item
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+  if (threadIdx.x == 0) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // prep's counter and status writes
+    if (*abort_flag) atomicOr(p.status, LLA_STATUS_TIMEOUT);
+    if constexpr (FUSE) {
+      // the last CTA to finish publishes this call's status bits (word 1) and clears
+      // word 0; otherwise the combine pass does it
+      __threadfence();
+      if (atomicAdd(&p.counters[(size_t)p.B * p.H], 1u) == gridDim.x - 1) {
+        __threadfence();
+        p.status[1] = atomicExch(&p.status[0], 0);
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 bool make_map(CUtensorMap* map, const void* base, int inner, int n_cap, int B, int box_inner,
@@ -1622,6 +2332,8 @@ int env_int(const char* name, int dflt) {
 struct TcPlan {
   bool ok = false;
   bool shared = false;    // LLA-2D kernel (G heads per item share each latent tile)
+  bool fform = false;     // phase-operand kernel (decode_tcf_kernel)
+  int ne = 2;             // its phase-tile buffers
   int G = 1, nst = 0, nst_v = 0, nacc = 1, nbuf_b = 2, S = 0, tps = 0;
   bool nope = false;      // decoupled RoPE: score operands carry a NoPE content column
   size_t ops_bytes = 0;   // workspace for the per-(b, h) operand images
@@ -1676,7 +2388,7 @@ uint32_t tc_layout(TcParams& p, int D, int G, int nst, int nst_v) {
   p.rope_off = o;            // float2 step[64], then uint2 phi[64]
   o += 64 * 8 * 2;
   p.bar_off = o;
-  o += (2 * nst + 2 * nst_v + 12) * 8;
+  o += (2 * nst + 2 * nst_v + 14) * 8;
   p.misc_off = o;
   o += 16;
   return o + 1024;
@@ -1732,10 +2444,77 @@ uint32_t tc2d_layout(TcParams& p, int D, int HP, int nst, int nst_v, int nbuf_b)
   p.rope_off = o;
   o += 64 * 8 * 2;
   p.bar_off = o;
-  o += (2 * nst + 2 * nst_v + 16) * 8;
+  o += (2 * nst + 2 * nst_v + 18) * 8;
   p.misc_off = o;
   o += 16;
   return o + 1024;
+}
+
+// Shared-memory layout of decode_tcf_kernel for (D, G, rings, image buffers, phase
+// buffers); r_k is a multiple of 16 and G r_v = 128.
+uint32_t tcf_layout(TcParams& p, int D, int G, int nst, int nst_v, int nbuf_b, int ne) {
+  auto al = [](uint32_t x, uint32_t a) { return (x + a - 1) / a * a; };
+  p.K_pad = p.r_k;
+  const int kw = G * p.r_k;                       // K latent columns of one item
+  p.box_k = kw % 64 == 0 ? 64 : 32;
+  p.nkb = kw / p.box_k;
+  p.swz = p.box_k == 64 ? 2 : 4;
+  p.kswz_mask = p.box_k == 64 ? 7 : 3;
+  p.box_bytes = kTile * p.box_k * 2;
+  p.tx_bytes = p.nkb * p.box_bytes;
+  p.st_bytes = al(p.tx_bytes, 1024);
+  p.N_v = p.r_v;
+  p.cvb = 64;                                     // V latent boxes: 64 dims, 128-byte rows
+  p.nvb = G * p.r_v / 64;
+  p.swz_v = 2;
+  p.vbox_bytes = kTile * 64 * 2;
+  p.tx_v = p.nvb * p.vbox_bytes;
+  p.stv_bytes = al(p.tx_v, 1024);
+  p.n_f = G * p.r_k + 16;
+  p.e_bytes = kTile * D * 2;
+  p.b_img_bytes = p.n_f * D * 2;
+  p.b_head_bytes = al(p.b_img_bytes, 1024);       // stride of the image buffers
+  p.nst = nst;
+  p.nst_v = nst_v;
+  p.nbuf_b = nbuf_b;
+  p.ne = ne;
+  uint32_t o = 0;
+  p.st_off = o;
+  o += nst * p.st_bytes;
+  p.stv_off = o;
+  o += nst_v * p.stv_bytes;
+  p.e_off = o;
+  o += ne * p.e_bytes;
+  p.b_off = o;
+  o += nbuf_b * p.b_head_bytes;
+  p.p_off = o;                                    // two weight buffers, 16 rows x 128 tokens
+  o += 2 * 4096;
+  p.red_off = o;
+  o = al(o + G * 4 * 4, 16);
+  p.comb_off = o;                                 // olat [128], misc [64]
+  o += (128 + 64) * 4;
+  p.ctx_off = o;
+  o += kCtxCache * 4;
+  p.rope_off = o;
+  o += 64 * 8 * 2;
+  p.bar_off = o;
+  o += (2 * nst + 2 * nst_v + 18) * 8;
+  p.misc_off = o;
+  o += 16;
+  return o + 1024;
+}
+
+// Whether the phase-operand kernel takes the shape: per head, RoPE over the whole
+// head of width 64 or 128, r_k of 16 or 32, and G = 128 / r_v of 2 or 4 heads per
+// item dividing H.  LLA_TC_FORM=u keeps such shapes on decode_tc_kernel.
+bool tcf_shape(const lla_cfg& c) {
+  const char* v = std::getenv("LLA_TC_FORM");
+  if (v && v[0] == 'u') return false;
+  if (c.mode != LLA_MODE_PER_HEAD || has_nope(c)) return false;
+  if (c.d_head != 64 && c.d_head != 128) return false;
+  if (c.r_k != 16 && c.r_k != 32) return false;
+  if (c.r_v != 32 && c.r_v != 64) return false;
+  return c.H % (128 / c.r_v) == 0;
 }
 
 TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
@@ -1752,6 +2531,39 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   // fit in 512 and whose shared-memory ring holds at least 2 stages; two score
   // buffers when they fit.
   int best_g = 0, best_nst = 0, best_nst_v = 0, best_nacc = 1;
+  if (tcf_shape(c)) {
+    // phase-operand kernel: three F buffers (3 n_f + 16 TMEM columns), then the most
+    // latent bytes in flight with two phase buffers and one image buffer (both can be
+    // forced: LLA_TCF_NE, LLA_TCF_NBUF)
+    const int G = 128 / c.r_v;
+    const int ne_f = env_int("LLA_TCF_NE", 0), nbuf_f = env_int("LLA_TCF_NBUF", 0);
+    for (int ne : {2, 1}) {
+      if (best_g || (ne_f && ne != ne_f)) continue;
+      for (int nbuf : {1, 2}) {
+        if (best_g || (nbuf_f && nbuf != nbuf_f) || (!nbuf_f && nbuf == 2)) continue;
+        TcParams p{};
+        p.r_k = c.r_k;
+        p.r_v = c.r_v;
+        uint32_t best_bytes = 0;
+        for (int nv = 8; nv >= 2; --nv)
+          for (int nk = 8; nk >= 2; --nk)
+            if (tcf_layout(p, c.d_head, G, nk, nv, nbuf, ne) <= kSmemLimit &&
+                nk * p.st_bytes + nv * p.stv_bytes > best_bytes) {
+              best_bytes = nk * p.st_bytes + nv * p.stv_bytes;
+              best_nst = nk;
+              best_nst_v = nv;
+            }
+        if (forced_nst && best_nst > forced_nst) best_nst = forced_nst;
+        if (forced_nst && best_nst_v > forced_nst) best_nst_v = forced_nst;
+        if (!best_bytes || best_nst < 2 || best_nst_v < 2) continue;
+        best_g = G;
+        best_nacc = 3;
+        pl.nbuf_b = nbuf;
+        pl.ne = ne;
+        pl.fform = true;
+      }
+    }
+  }
   if (c.mode == LLA_MODE_2D) {
     // HP heads per item share each latent tile: the largest HP whose operands fit,
     // double-buffered when possible; three one-head score buffers when TMEM allows.
@@ -1787,7 +2599,7 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
     }
   }
   for (int G : {4, 2, 1}) {
-    if (pl.shared) break;
+    if (pl.shared || pl.fform) break;
     if (c.H % G) continue;
     if (forced_g && G != forced_g) continue;
     int nacc = 0;
@@ -1861,7 +2673,8 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   pl.tps = (n_tiles + best_s - 1) / best_s;
   pl.S = (n_tiles + pl.tps - 1) / pl.tps;
   const size_t K_pad = (c.r_k + 15) / 16 * 16;
-  pl.ops_bytes = (size_t)B * c.H * ((size_t)D * K_pad * 2 + (size_t)D * 32);
+  pl.ops_bytes = pl.fform ? (size_t)B * (c.H / pl.G) * ((size_t)pl.G * c.r_k + 16) * c.d_head * 2
+                          : (size_t)B * c.H * ((size_t)D * K_pad * 2 + (size_t)D * 32);
   pl.nope = nope;
   pl.ok = true;
   return pl;
@@ -1929,6 +2742,60 @@ cudaError_t launch_tc_nope(int G, bool shared, const CUtensorMap& mk, const CUte
   }
 }
 
+template <int D, int G, int KP>
+cudaError_t launch_tcf_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
+                         uint32_t smem, int grid, cudaStream_t s) {
+  void (*kern)(CUtensorMap, CUtensorMap, TcParams) =
+      p.fuse_combine ? decode_tcf_kernel<D, G, KP, true> : decode_tcf_kernel<D, G, KP, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // programmatic dependent launch after the prep kernel: the producers wait for its
+  // grid only before the first operand-image load
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
+}
+
+cudaError_t launch_tcf(int D, int G, int KP, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
+#define LLA_TCF(DD, GG, KK) \
+  if (D == DD && G == GG && KP == KK) return launch_tcf_t<DD, GG, KK>(mk, mv, p, smem, grid, s)
+  LLA_TCF(128, 4, 16);
+  LLA_TCF(128, 4, 32);
+  LLA_TCF(128, 2, 16);
+  LLA_TCF(128, 2, 32);
+  LLA_TCF(64, 4, 16);
+  LLA_TCF(64, 4, 32);
+  LLA_TCF(64, 2, 16);
+  LLA_TCF(64, 2, 32);
+#undef LLA_TCF
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_prep_f(const DecodeArgs& a, const TcParams& p, int G, cudaStream_t s) {
+  dim3 grid((unsigned)a.H, (unsigned)a.B);
+  unsigned char* ob = const_cast<unsigned char*>(p.ops_b);
+  if (a.d == 128)
+    decode_prep_f_kernel<128><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t,
+                                                   a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
+                                                   p.b_img_bytes, ob, a.status, a.counters);
+  else if (a.d == 64)
+    decode_prep_f_kernel<64><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t,
+                                                  a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
+                                                  p.b_img_bytes, ob, a.status, a.counters);
+  else
+    return cudaErrorNotSupported;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prep(const DecodeArgs& a, const TcParams& p, cudaStream_t s) {
   const int ns = a.rd < a.d ? a.rd + 16 : a.d;      // image rows per head
   const int chunks = ns * p.K_pad / 8;
@@ -1987,8 +2854,9 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.r_v = a.r_v;
   // At least 120 KB so that two CTAs never share an SM (each may hold all of TMEM).
   const int ns = pl.nope ? a.rd + 16 : a.d;   // score columns per head
-  uint32_t smem = pl.shared ? tc2d_layout(p, ns, pl.G, pl.nst, pl.nst_v, pl.nbuf_b)
-                            : tc_layout(p, ns, pl.G, pl.nst, pl.nst_v);
+  uint32_t smem = pl.fform    ? tcf_layout(p, a.d, pl.G, pl.nst, pl.nst_v, pl.nbuf_b, pl.ne)
+                 : pl.shared ? tc2d_layout(p, ns, pl.G, pl.nst, pl.nst_v, pl.nbuf_b)
+                             : tc_layout(p, ns, pl.G, pl.nst, pl.nst_v);
   if (smem < 120u * 1024u) smem = 120u * 1024u;
   p.B = a.B;
   p.n_cap = a.n_cap;
@@ -1998,9 +2866,9 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.n_items = a.B * p.HG * pl.S;
   p.rope_max_pos = a.rope_max_pos;
   p.nacc = pl.nacc;
-  p.acc_cols = pl.shared ? ns : pl.G * ns;
+  p.acc_cols = pl.fform ? p.n_f : pl.shared ? ns : pl.G * ns;
   p.v_col0 = p.nacc * p.acc_cols;
-  const int v_cols = pl.shared ? p.m_v * p.n_p : pl.G * p.N_v;
+  const int v_cols = pl.fform ? 16 : pl.shared ? p.m_v * p.n_p : pl.G * p.N_v;
   int cols = 32;
   while (cols < p.v_col0 + v_cols) cols <<= 1;
   p.tmem_cols = cols;
@@ -2043,6 +2911,20 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.poll = env_int("LLA_TC_POLL", 1);
   p.lat_hk = (int)a.lat_head_k;
   p.lat_hv = (int)a.lat_head_v;
+  if (pl.fform) {
+    // K latents of an item: the G heads' r_k columns side by side (128- or 64-byte
+    // rows); V latents: 64-dim boxes with 128-byte rows
+    if (!make_map(&mk, a.ck, (int)a.lat_tok_k, a.n_cap, a.B, p.box_k, swz) ||
+        !make_map(&mv, a.cv, (int)a.lat_tok_v, a.n_cap, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorNotSupported;
+    const int sms = sm_count();
+    cudaError_t pe = launch_prep_f(a, p, pl.G, s);
+    if (pe != cudaSuccess) return pe;
+    const int grid = p.n_items < sms ? p.n_items : sms;
+    cudaError_t e = launch_tcf(a.d, pl.G, a.r_k, mk, mv, p, smem, grid, s);
+    if (e == cudaSuccess && !p.fuse_combine) e = launch_combine(a, s);
+    return e;
+  }
   if (!make_map(&mk, a.ck, (int)a.lat_tok_k, a.n_cap, a.B, p.box_k, swz) ||
       !make_map(&mv, a.cv, (int)a.lat_tok_v, a.n_cap, a.B, p.cvb,
                 p.cvb == 64   ? CU_TENSOR_MAP_SWIZZLE_128B

@@ -162,3 +162,24 @@ def test_forced_split_count_is_clamped(monkeypatch):
     short = lla.lib.lla_decode_workspace_bytes(c, B, 300)    # 3 tiles
     monkeypatch.setenv("LLA_TC_SPLITS", "3")
     assert short == lla.lib.lla_decode_workspace_bytes(c, B, 300)
+
+
+def test_phase_operand_kernel_workspace():
+    """Per-head shapes with r_k in {16, 32} and G = 128 / r_v heads per item run on
+    the phase-operand kernel, whose operand images are one [G r_k + 16, d] bf16 image
+    per (sequence, head group); LLA_TC_FORM=u keeps them on the per-head kernel, whose
+    images are per (sequence, head)."""
+    import os
+    cfg = lla.Cfg(4, 16, 128, 16, 32)
+    c = ctypes.byref(cfg.c())
+    B, n = 256, 4097
+    ws_f = lla.lib.lla_decode_workspace_bytes(c, B, n)
+    os.environ["LLA_TC_FORM"] = "u"
+    try:
+        ws_u = lla.lib.lla_decode_workspace_bytes(c, B, n)
+    finally:
+        del os.environ["LLA_TC_FORM"]
+    img_f = B * (16 // 4) * (4 * 16 + 16) * 128 * 2
+    img_u = B * 16 * (128 * 16 * 2 + 128 * 32)
+    assert ws_u - ws_f == img_u - img_f
+    assert lla.decode_launches(cfg, B, n) == 2

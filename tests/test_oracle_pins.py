@@ -243,6 +243,97 @@ def test_eckart_young_and_monotone_error():
     assert cal[2] < 1e-2 * cal[0]
 
 
+def test_2d_svd_codec_full_rank_is_exact_and_slice_order_matters():
+    """LLA-2D branch of svd_codec and loop_slices (close reading §二.4, §二.6; gist.science
+    "Training und Initialisierung", "LLA-2D-Variante"): with r = T H d the SVD basis of
+    the (t, h, i)-ordered calibration rows is a full orthonormal basis, so encoding and
+    then rebuilding with the (t, h) slice returns x_{t,h} exactly.  Slicing the rows in
+    (h, t) order instead (a transposed reshape) does not."""
+    g = synth.rng(41)
+    T, H, d = 2, 3, 4                             # width T H d = 24
+    W = T * H * d
+    cfg = O.Cfg(T, H, d, W, W, O.MODE_2D)
+    model = synth.trajectory_model(g, T, H, d, R=5, shared=True)
+    cal_k = synth.sample_trajectories(g, model, 400)
+    cal_v = synth.sample_trajectories(g, model, 400)
+    codec = O.svd_codec(cfg, cal_k, cal_v)
+    assert codec.W_down_k.shape == (W, W) and codec.W_up_k.shape == (T, H, d, W)
+    np.testing.assert_allclose(codec.W_down_k.T @ codec.W_down_k, np.eye(W), atol=1e-12)
+    x = synth.sample_trajectories(g, model, 10)
+    ck, cv = O.encode_tokens(cfg, codec, x, x)
+    wrong_order = codec.W_down_k.reshape(H, T, d, W)
+    worst_wrong = 0.0
+    for t in range(T):
+        for h in range(H):
+            mu = O.mu_t(cfg, codec.mu_k, t, h)
+            rec = O.reconstruct(ck, O.w_up_t(cfg, codec.W_up_k, t, h), mu)
+            np.testing.assert_allclose(rec, x[:, t, h], atol=1e-12)
+            np.testing.assert_allclose(O.reconstruct(cv, O.w_up_t(cfg, codec.W_up_v, t, h),
+                                                     O.mu_t(cfg, codec.mu_v, t, h)),
+                                       x[:, t, h], atol=1e-12)
+            bad = O.reconstruct(ck, wrong_order[h, t], mu)
+            worst_wrong = max(worst_wrong, np.abs(bad - x[:, t, h]).max())
+    assert worst_wrong > 0.1
+
+
+def test_2d_eckart_young_and_monotone_error():
+    """LLA-2D codec by SVD: the calibration error summed over every (t, h) rebuild equals
+    the discarded spectrum, so it falls monotonically with r (held-out error too, on the
+    seeded low-rank-plus-noise trajectories shared across heads)."""
+    g = synth.rng(43)
+    T, H, d = 2, 2, 6
+    W = T * H * d
+    model = synth.trajectory_model(g, T, H, d, R=4, shared=True)
+    X = synth.sample_trajectories(g, model, 300)
+    Xh = synth.sample_trajectories(g, model, 300)
+    cal, held = [], []
+    for r in range(1, W + 1, 2):
+        mu, Wd, sigma = O.svd_init(X.reshape(300, W), r)
+        W_up = O.loop_slices(Wd, T, d, H)
+        assert W_up.shape == (T, H, d, r)
+        cfg = O.Cfg(T, H, d, r, r, O.MODE_2D)
+        for data, acc in ((X, cal), (Xh, held)):
+            c = O.encode(data.reshape(len(data), W), mu, Wd)
+            err = 0.0
+            for t in range(T):
+                for h in range(H):
+                    rec = O.reconstruct(c, W_up[t, h], O.mu_t(cfg, mu, t, h))
+                    err += ((data[:, t, h] - rec) ** 2).sum()
+            acc.append(err)
+        assert cal[-1] == pytest.approx((sigma[r:] ** 2).sum(), rel=1e-9, abs=1e-9)
+    assert all(a >= b - 1e-9 for a, b in zip(cal, cal[1:]))
+    assert all(a >= b - 1e-9 for a, b in zip(held, held[1:]))
+    assert cal[2] < 1e-2 * cal[0]      # rank 4 plus noise: captured once r >= 5
+
+
+def test_2d_svd_codec_error_is_the_discarded_spectrum():
+    """The whole LLA-2D codec path (svd_codec on [N, T, H, d] calibration tokens,
+    encode_tokens, the (t, h) slices of W_up and mu) at ranks below full: the
+    calibration error over every (t, h) rebuild equals the sum of the discarded
+    squared singular values of the centred (t, h, i)-ordered calibration matrix, as
+    numpy's SVD gives them.  A codec built in another concatenation order, or with a
+    mis-sliced mean, misses it."""
+    g = synth.rng(47)
+    T, H, d = 2, 3, 4
+    W = T * H * d
+    model = synth.trajectory_model(g, T, H, d, R=6, shared=True)
+    N = 300
+    X = synth.sample_trajectories(g, model, N)
+    flat = X.reshape(N, W)                               # (t, h, i) order, [CR] §二.6
+    sigma = np.linalg.svd(flat - flat.mean(0), compute_uv=False)
+    for r in (3, 6, 11):
+        cfg = O.Cfg(T, H, d, r, r, O.MODE_2D)
+        codec = O.svd_codec(cfg, X, X)
+        ck, _ = O.encode_tokens(cfg, codec, X, X)
+        err = 0.0
+        for t in range(T):
+            for h in range(H):
+                rec = O.reconstruct(ck, O.w_up_t(cfg, codec.W_up_k, t, h),
+                                    O.mu_t(cfg, codec.mu_k, t, h))
+                err += ((X[:, t, h] - rec) ** 2).sum()
+        assert err == pytest.approx((sigma[r:] ** 2).sum(), rel=1e-9, abs=1e-9)
+
+
 # --------------------------------------------------------------------------- attention
 
 def brute_force(q, K, V, pos, ks, vs, qpos, base):

@@ -5,6 +5,8 @@ relative error per (b, h); encoded latents within 1e-2 of the latent's L2 norm
 (against the unrounded fp64 value); RoPE table within 1e-7 absolute; status
 bits and bookkeeping exact.
 """
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -89,6 +91,38 @@ def test_encode_matches_oracle(cfg, n_tok, path, monkeypatch):
     assert np.all(ck.float().cpu().numpy()[untouched] == 0)
 
 
+def test_encode_deep_loop_full_width_sampled():
+    """The deep-loop codec at its full width (T = 32, H = 8, d = 96: 3072 entries per
+    head's latent) on the tensor-core encode, 4096 tokens in scattered slots, sampled
+    rows of every head against the oracle."""
+    w = synth.WORKLOADS["deeploop_32x_T32_H8_d96_r64_128_B16_n32768"]
+    cfg = O.Cfg(w.T, w.H, w.d, w.r_k, w.r_v, w.mode)
+    cod = synth.workload_codec(w)
+    codec = O.Codec(*(cod[k].astype(np.float64) for k in
+                      ("W_down_k", "W_down_v", "W_up_k", "W_up_v", "mu_k", "mu_v")))
+    packed = lla.codec_pack(lib_cfg(cfg), *(torch.from_numpy(cod[k]).cuda() for k in
+                                            ("W_down_k", "W_down_v", "W_up_k", "W_up_v",
+                                             "mu_k", "mu_v")))
+    n_tok, n_slots = 4096, 5000
+    g = synth.rng(4242)
+    model = synth.trajectory_model(g, w.T, w.H, w.d, w.R, gamma=w.gamma)
+    xk = O.bf16_round(synth.sample_trajectories(g, model, n_tok))
+    xv = O.bf16_round(synth.sample_trajectories(g, model, n_tok))
+    slot = g.permutation(n_slots)[:n_tok]
+    ck = torch.zeros((n_slots, w.H, w.r_k), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros((n_slots, w.H, w.r_v), dtype=torch.bfloat16, device="cuda")
+    lla.encode(lib_cfg(cfg), packed, bf16_tensor(xk), bf16_tensor(xv),
+               torch.from_numpy(slot.astype(np.int64)).cuda(), ck, cv)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, 127, 128, n_tok - 1], g.integers(0, n_tok, 60)]))
+    want_k, want_v = O.encode_tokens(cfg, codec, xk[rows], xv[rows])
+    got_k = ck.double().cpu().numpy()[slot[rows]]
+    got_v = cv.double().cpu().numpy()[slot[rows]]
+    for got, want in ((got_k, want_k), (got_v, want_v)):
+        err = np.abs(got - want).max(-1) / np.linalg.norm(want, axis=-1)
+        assert err.max() <= LATENT_TOL, err.max()
+
+
 def test_encode_out_of_range_slot_sets_status_and_skips():
     cfg = O.Cfg(4, 2, 64, 8, 16)
     case = decode_case(cfg, 1, 4, seed=3)
@@ -124,6 +158,16 @@ SMALL = [
     (O.Cfg(4, 6, 96, 48, 160, O.MODE_2D), 2, 260, [260, 131], {}),
     (O.Cfg(2, 3, 32, 16, 24, O.MODE_2D), 3, 140, [140, 1, 0], {}),
     (O.Cfg(4, 8, 64, 32, 64, O.MODE_2D), 2, 390, None, {"positions": "random", "q_scale": 20.0}),
+    # phase-operand kernel (per head, r_k 16 or 32, G = 128 / r_v heads per item):
+    # the 21.3x shape, two head groups with random positions and a sharp softmax,
+    # d 64 with two heads per item, ragged and empty contexts, r_k 32, a random codec,
+    # and one sequence long enough for several context splits (combine pass)
+    (O.Cfg(4, 4, 128, 16, 32), 2, 600, [600, 257], {}),
+    (O.Cfg(4, 8, 128, 16, 32), 2, 300, None, {"positions": "random", "q_scale": 20.0}),
+    (O.Cfg(4, 4, 64, 32, 64), 3, 300, [300, 129, 1], {}),
+    (O.Cfg(4, 4, 128, 32, 32), 2, 400, [400, 0], {"q_scale": 25.0}),
+    (O.Cfg(4, 4, 64, 16, 32), 2, 260, None, {"codec": "random"}),
+    (O.Cfg(4, 4, 128, 16, 32), 1, 2000, None, {}),
 ]
 
 
@@ -137,6 +181,55 @@ def test_decode_matches_oracle_small(spec):
         want = expected(case, t)
         err = rel_err(got, want)
         assert np.isfinite(got).all()
+        assert err.max() <= ATTN_TOL, (t, err.max())
+    assert lla.decode_status(dev.ws) == 0
+
+
+# The CUDA-core decode kernel: the path for shapes the tensor-core plan refuses (here
+# d 128 with r_k = r_v = 256, whose K and V rings do not fit in shared memory), and
+# the LLA_DECODE_PATH=cuda_core variant of every small case.
+CUDA_CORE_ONLY = [
+    (O.Cfg(4, 2, 128, 256, 256), 2, 300, [300, 131], {}),
+    (O.Cfg(2, 2, 128, 256, 256, O.MODE_2D), 1, 200, None, {"q_scale": 10.0}),
+]
+
+
+def test_tensor_core_plan_refuses_the_cuda_core_shapes():
+    for cfg, B, n_cap, _, _ in CUDA_CORE_ONLY:
+        # partial kernel + combine: the CUDA-core plan
+        assert lla.decode_launches(lib_cfg(cfg), B, n_cap) == 2
+        ws = lla.lib.lla_decode_workspace_bytes(ctypes.byref(lib_cfg(cfg).c()), B, n_cap)
+        assert ws > 0
+
+
+@pytest.mark.parametrize("spec", SMALL + CUDA_CORE_ONLY,
+                         ids=lambda s: f"T{s[0].T}H{s[0].H}d{s[0].d}r{s[0].r_k}_{s[0].r_v}m{s[0].mode}B{s[1]}n{s[2]}")
+def test_cuda_core_decode_matches_oracle(spec, monkeypatch):
+    monkeypatch.setenv("LLA_DECODE_PATH", "cuda_core")
+    cfg, B, n_cap, ctx, kw = spec
+    case = decode_case(cfg, B, n_cap, seed=300 + n_cap, ctx_len=ctx, **kw)
+    dev = DeviceCase(case)
+    for t in (0, cfg.T - 1):
+        got = dev.decode(t)
+        err = rel_err(got, expected(case, t))
+        assert np.isfinite(got).all()
+        assert err.max() <= ATTN_TOL, (t, err.max())
+    assert lla.decode_status(dev.ws) == 0
+
+
+@pytest.mark.parametrize("spec", [s for s in SMALL if s[0].mode == O.MODE_PER_HEAD
+                                  and s[0].r_k in (16, 32) and s[0].r_v in (32, 64)
+                                  and s[0].H % (128 // s[0].r_v) == 0 and s[0].d in (64, 128)],
+                         ids=lambda s: f"T{s[0].T}H{s[0].H}d{s[0].d}r{s[0].r_k}_{s[0].r_v}B{s[1]}n{s[2]}")
+def test_per_head_kernel_on_phase_operand_shapes(spec, monkeypatch):
+    """LLA_TC_FORM=u runs the shapes of the phase-operand kernel on the per-head
+    tensor-core kernel instead: both against the oracle."""
+    monkeypatch.setenv("LLA_TC_FORM", "u")
+    cfg, B, n_cap, ctx, kw = spec
+    case = decode_case(cfg, B, n_cap, seed=100 + n_cap, ctx_len=ctx, **kw)
+    dev = DeviceCase(case)
+    for t in (0, cfg.T - 1):
+        err = rel_err(dev.decode(t), expected(case, t))
         assert err.max() <= ATTN_TOL, (t, err.max())
     assert lla.decode_status(dev.ws) == 0
 
