@@ -1712,30 +1712,30 @@ __global__ void __launch_bounds__(128) decode_prep_f_kernel(
   }
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) {
-  const __nv_bfloat162 b = __floats2bfloat162_rn(v.x, v.y);   // .x in the low half
-  uint32_t u;
-  memcpy(&u, &b, 4);
-  return u;
-}
-
 // bf16 pair (low half first) -> two floats
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// D: head width; G: heads per item (G r_v = 128, the M of the V MMA); KP: r_k.
-// Warps as in decode_tc_kernel: 0 K latent producer (and each item's operand image),
-// 1 F MMA issuer, 2..9 epilogue (two warpgroups: warpgroup w owns heads
-// [w G/2, (w + 1) G/2) of the item for scores and softmax, and half of the RoPE pairs
-// of the phase tiles it writes), 10 V latent producer, 11 V MMA issuer.
-template <int D, int G, int KP, bool FUSE>
-__global__ void __launch_bounds__(kThreads, 1)
+// Warps of decode_tcf_kernel: 0 K latent producer (and each item's operand image),
+// 1 F MMA issuer, 2 .. 17 epilogue (four warpgroups: warpgroup w owns head w of the
+// item for scores, softmax and weights, and a quarter of the RoPE pairs of the phase
+// tiles it writes), 18 V latent producer, 19 V MMA issuer.
+constexpr int kGF = 4;                          // heads per item (G r_v = 128)
+constexpr int kEpiWGF = 4;
+constexpr int kEpiThreadsF = 128 * kEpiWGF;
+constexpr int kEpiWarpsF = kEpiThreadsF / 32;
+constexpr int kThreadsF = 64 + kEpiThreadsF + 64;
+constexpr int kVProdWarpF = 2 + kEpiWarpsF, kVMmaWarpF = 3 + kEpiWarpsF;
+
+// D: head width; KP: r_k (16 or 32).  r_v = 32, so the G = 4 heads' V latents fill
+// the M = 128 of the transposed V MMA.
+template <int D, int KP, bool FUSE>
+__global__ void __launch_bounds__(kThreadsF, 1)
     decode_tcf_kernel(const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
-  constexpr int HW = G / kEpiWG;             // heads per epilogue warpgroup
-  constexpr int WG_PAIRS = D / 2 / kEpiWG;   // RoPE pairs of a token row each warpgroup writes
-  constexpr int NBIAS = 2 * G <= 8 ? 8 : 16; // bias columns read (hi, lo of every head)
-  static_assert(HW >= 1 && WG_PAIRS % 4 == 0 && KP % 16 == 0, "shape");
+  constexpr int G = kGF;
+  constexpr int WG_PAIRS = D / 2 / kEpiWGF;  // RoPE pairs of a token row each warpgroup writes
+  static_assert(WG_PAIRS % 4 == 0 && KP % 16 == 0, "shape");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -1756,11 +1756,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
+  // hand-off waits: polled (the default, LLA_TC_POLL=1) or suspending
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return p.poll ? mbar_wait_poll(bar, parity, abort_flag) : mbar_wait(bar, parity, abort_flag);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.nst; ++s) {
       mbar_init(&full_k[s], 1);
-      mbar_init(&empty_k[s], kEpiWarps);
+      mbar_init(&empty_k[s], kEpiWarpsF);
     }
     for (int s = 0; s < p.nst_v; ++s) {
       mbar_init(&full_v[s], 1);
@@ -1768,13 +1772,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 3; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiWarps);
+      mbar_init(&tempty[a], kEpiWarpsF);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&efull[a], kEpiWarps);
+      mbar_init(&efull[a], kEpiWarpsF);
       mbar_init(&bfull[a], 1);
       mbar_init(&bempty[a], 1);
-      mbar_init(&pfull[a], kEpiWarps);
+      mbar_init(&pfull[a], kEpiWarpsF);
       mbar_init(&pempty[a], 1);
     }
     mbar_init(&drain[0], 1);
@@ -1786,11 +1790,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, p.tmem_cols);
     tmem_relinquish();
   }
-  if (warp >= 2 && warp < 2 + kEpiWarps) {
+  if (warp >= 2 && warp < 2 + kEpiWarpsF) {
     const int et = threadIdx.x - 64;
     if (ctx_s) {
       int* cs = reinterpret_cast<int*>(sm + p.ctx_off);
-      for (int b = et; b < p.B; b += kEpiThreads) {
+      for (int b = et; b < p.B; b += kEpiThreadsF) {
         int n = p.ctx_len[b];
         if (n < 0 || n > p.n_cap) {
           if (blockIdx.x == 0) atomicOr(p.status, LLA_STATUS_CTX_RANGE);
@@ -1804,7 +1808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<uint2*>(sm + p.rope_off + 512)[et] = make_uint2(p.phi_lo[et], p.phi_hi[et]);
     }
     // both weight buffers start zero: rows >= 2G are never written
-    for (int idx = et; idx < 2 * 4096 / 4; idx += kEpiThreads)
+    for (int idx = et; idx < 2 * 4096 / 4; idx += kEpiThreadsF)
       reinterpret_cast<uint32_t*>(sm + p.p_off)[idx] = 0u;
     fence_proxy_async_smem();
   }
@@ -1813,7 +1817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0 || warp == kVProdWarp) {
+  if (warp == 0 || warp == kVProdWarpF) {
     // ------------------------------------------------------------ TMA producers
     if (lane == 0) {
       const bool kside = warp == 0;
@@ -1841,7 +1845,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int k = 0; k < r.ntiles; ++k, ++it) {
           const uint32_t stage = it % nst, ph = (it / nst) & 1u;
-          if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {
+          if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {   // producers suspend
             ok = false;
             break;
           }
@@ -1894,14 +1898,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const ItemRange r = item_range(p, ctx_s, item, false);
         if (r.ntiles == 0) continue;
         const uint32_t buf = jn % p.nbuf_b, bph = (jn / p.nbuf_b) & 1u;
-        if (!mbar_wait(&bfull[buf], bph, abort_flag)) break;
+        if (!wait(&bfull[buf], bph)) break;
         ++jn;
         const uint32_t b_base = b_base0 + buf * p.b_head_bytes;
         for (int k = 0; k < r.ntiles; ++k, ++it) {
           const uint32_t e = it % p.ne, eph = (it / p.ne) & 1u;
           const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
-          if (!mbar_wait(&efull[e], eph, abort_flag) ||
-              !mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
+          if (!wait(&efull[e], eph) || !wait(&tempty[acc], aph ^ 1u)) {
             ok = false;
             break;
           }
@@ -1922,7 +1925,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_drain(&drain[0]);
     }
     __syncwarp();
-  } else if (warp == kVMmaWarp) {
+  } else if (warp == kVMmaWarpF) {
     // ------------------------------------------------------------ V MMA issuer
     // D_v^T (G r_v = 128 latent dims x 16) (+)= C_v^T (128 x 128 tokens, MN-major A,
     // two 64-dim boxes) x P^T (128 tokens x 16 weight rows, K-major B).
@@ -1937,8 +1940,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < r.ntiles; ++k, ++it) {
           const uint32_t pb = it & 1u;
           const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
-          if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag) ||
-              !mbar_wait(&full_v[vs], vph, abort_flag)) {
+          if (!wait(&pfull[pb], (it >> 1) & 1u) || !wait(&full_v[vs], vph)) {
             ok = false;
             break;
           }
@@ -1961,7 +1963,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;
-    const int wgi = (warp - 2) >> 2;          // warpgroup: heads [wgi HW, (wgi + 1) HW)
+    const int wgi = (warp - 2) >> 2;          // warpgroup = head of the item
     const int sub = warp & 3;                 // TMEM sub-partition of this warp
     const int row = sub * 32 + lane;          // token row of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
@@ -1972,9 +1974,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Phase tiles: the RoPE factors conj(e^{i p theta_i}) of this warpgroup's pairs at
     // this thread's token row of the last tile written, advanced by one complex
     // product when the next tile's token sits a tile further on (as in
-    // decode_tc_kernel), and a cursor over the tiles still to write.
+    // decode_tc_kernel), and a cursor over the tiles still to write.  The position of
+    // the next tile to write is loaded one tile before it is used.
     TileCursor ec;
     cursor_first(p, ctx_s, ec);
+    bool e_more = ec.valid;                   // a phase tile is left to write
+    int pos_pref = cursor_pos(p, ec, row);    // its raw position at this thread's row
+    cursor_next(p, ctx_s, ec);
     float2 ef[WG_PAIRS];
     int pos_cur = kNoPos, run = 0;
     const float2* step_s = reinterpret_cast<const float2*>(sm + p.rope_off) + wgi * WG_PAIRS;
@@ -2003,56 +2009,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int q = 0; q < WG_PAIRS; ++q) ef[q] = make_float2(1.f, 0.f);
     uint32_t ie = 0;   // phase tiles written
-    // Write this thread's row of the next phase tile into buffer ie % ne: entries
+    // This thread's row of the next phase tile into buffer ie % ne: entries
     // (2i, 2i + 1) = (cos, -sin) of pair i, 128-byte swizzled K-major rows.
     auto write_e = [&]() {
-      advance_rope(cursor_pos(p, ec, row));
+      advance_rope(pos_pref);
       unsigned char* eb = sm + p.e_off + (ie % p.ne) * p.e_bytes;
 #pragma unroll
       for (int c = 0; c < WG_PAIRS / 4; ++c) {
         const int pair0 = wgi * WG_PAIRS + c * 4;
         const int blk = pair0 >> 5, ch = (pair0 >> 2) & 7;
         uint4 v;
-        v.x = pack_bf16x2(ef[c * 4 + 0]);
-        v.y = pack_bf16x2(ef[c * 4 + 1]);
-        v.z = pack_bf16x2(ef[c * 4 + 2]);
-        v.w = pack_bf16x2(ef[c * 4 + 3]);
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(ef[c * 4 + 0].x, ef[c * 4 + 0].y);
+        __nv_bfloat162 b1 = __floats2bfloat162_rn(ef[c * 4 + 1].x, ef[c * 4 + 1].y);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(ef[c * 4 + 2].x, ef[c * 4 + 2].y);
+        __nv_bfloat162 b3 = __floats2bfloat162_rn(ef[c * 4 + 3].x, ef[c * 4 + 3].y);
+        memcpy(&v.x, &b0, 4);
+        memcpy(&v.y, &b1, 4);
+        memcpy(&v.z, &b2, 4);
+        memcpy(&v.w, &b3, 4);
         *reinterpret_cast<uint4*>(eb + blk * (kTile * 128) + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&efull[ie % p.ne]);
+      e_more = ec.valid;
+      pos_pref = cursor_pos(p, ec, row);      // used by the next call
       cursor_next(p, ctx_s, ec);
       ++ie;
     };
-    for (int k = 0; k < p.ne && ec.valid; ++k) write_e();
+    for (int k = 0; k < p.ne && e_more; ++k) write_e();
 
     uint32_t it = 0;
     bool aborted = false;
     for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
       const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
-      float m_ref[HW], l_part[HW];
-#pragma unroll
-      for (int hh = 0; hh < HW; ++hh) {
-        m_ref[hh] = -INFINITY;
-        l_part[hh] = 0.f;
-      }
+      float m_ref = -INFINITY, l_part = 0.f;   // head wgi of the item
       if constexpr (FUSE) {
-        // fused finish, set up while the tiles stream: the in-flight scores' partial
-        // dot products q . k_self (per warp of warpgroup 0), and the heads' W_up,v rows
-        // into L2, kept there ahead of the latent stream
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const size_t bh = (size_t)r.b * p.H + r.hg * G + g;
-          if (wgi == 0) {
-            const float qk = row < p.d ? __ldg(p.q + bh * p.d + row) * __ldg(p.k_self + bh * p.d + row) : 0.f;
-            const float sdot = warp_sum_f(qk);
-            if (lane == 0) misc[8 + g * 4 + sub] = sdot;
-          }
-          const char* wrow = reinterpret_cast<const char*>(p.wupv_t + (size_t)(r.hg * G + g) * p.d * p.r_v);
-          for (int off = et * 128; off < p.d * p.r_v * 4; off += kEpiThreads * 128)
-            asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wrow + off));
-        }
+        // fused finish, set up while the tiles stream: the in-flight score's partial
+        // dot products q . k_self (per warp), and the head's W_up,v rows into L2,
+        // kept there ahead of the latent stream
+        const size_t bh = (size_t)r.b * p.H + r.hg * G + wgi;
+        const float qk = row < p.d ? __ldg(p.q + bh * p.d + row) * __ldg(p.k_self + bh * p.d + row) : 0.f;
+        const float sdot = warp_sum_f(qk);
+        if (lane == 0) misc[8 + wgi * 4 + sub] = sdot;
+        const char* wrow = reinterpret_cast<const char*>(p.wupv_t + (size_t)(r.hg * G + wgi) * p.d * p.r_v);
+        for (int off = row * 128; off < p.d * p.r_v * 4; off += 128 * 128)
+          asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wrow + off));
       }
       for (int k = 0; k < r.ntiles; ++k, ++it) {
         const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
@@ -2061,115 +2063,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cnt = min(kTile, r.tok_end - t0);
         const bool valid = row < cnt;
 
-        bool ok = mbar_wait(&tfull[acc], aph, abort_flag);
+        bool ok = wait(&tfull[acc], aph);
         tc_fence_after();
-        float f[HW][KP];
-        float fb[NBIAS];
+        float f[KP];
+        float fb[2];
+        {
+          const uint32_t col = tmem_base + lane_addr + acc * p.n_f;
 #pragma unroll
-        for (int hh = 0; hh < HW; ++hh) {
-          const uint32_t col = tmem_base + lane_addr + acc * p.n_f + (wgi * HW + hh) * KP;
-#pragma unroll
-          for (int c = 0; c < KP / 16; ++c) tmem_ld16(col + c * 16, &f[hh][c * 16]);
+          for (int c = 0; c < KP / 16; ++c) tmem_ld16(col + wgi * KP + c * 16, &f[c * 16]);
+          tmem_ld2(col + G * KP + 2 * wgi, fb);
         }
-        if constexpr (NBIAS == 8)
-          tmem_ld8(tmem_base + lane_addr + acc * p.n_f + G * KP, fb);
-        else
-          tmem_ld16(tmem_base + lane_addr + acc * p.n_f + G * KP, fb);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
-        // one phase buffer: the next tile's E goes in as soon as F of this one is out
-        if (p.ne == 1 && ec.valid) write_e();
 
-        // s = sum_m c_m F_m + F_M for each of this warpgroup's heads, with this token
-        // row's latents read from the swizzled K tile
-        ok = ok && mbar_wait(&full_k[stage], kph, abort_flag);
-        float s[HW];
+        // s = sum_m c_m F_m + F_M for head wgi, with this token row's latents read
+        // from the swizzled K tile
+        ok = ok && wait(&full_k[stage], kph);
+        float sc;
         {
           const unsigned char* st = sm + p.st_off + stage * p.st_bytes;
           const uint32_t row_bytes = (uint32_t)p.box_k * 2;
+          const int e0 = wgi * KP;                         // first latent column of the head
+          const unsigned char* bx = st + (e0 / p.box_k) * p.box_bytes;
+          const uint32_t c0 = (uint32_t)(e0 % p.box_k) * 2 / 16;
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-          for (int hh = 0; hh < HW; ++hh) {
-            const int e0 = (wgi * HW + hh) * KP;           // first latent column of the head
-            const unsigned char* bx = st + (e0 / p.box_k) * p.box_bytes;
-            const uint32_t c0 = (uint32_t)(e0 % p.box_k) * 2 / 16;
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int cc = 0; cc < KP / 8; ++cc) {
-              const uint32_t L = row * row_bytes + (c0 + cc) * 16;
-              const uint4 w = *reinterpret_cast<const uint4*>(
-                  bx + (L ^ (((L >> 7) & (uint32_t)p.kswz_mask) << 4)));
-              const float* fr = &f[hh][cc * 8];
-              a0 = fmaf(bf_lo(w.x), fr[0], a0);
-              a1 = fmaf(bf_hi(w.x), fr[1], a1);
-              a0 = fmaf(bf_lo(w.y), fr[2], a0);
-              a1 = fmaf(bf_hi(w.y), fr[3], a1);
-              a0 = fmaf(bf_lo(w.z), fr[4], a0);
-              a1 = fmaf(bf_hi(w.z), fr[5], a1);
-              a0 = fmaf(bf_lo(w.w), fr[6], a0);
-              a1 = fmaf(bf_hi(w.w), fr[7], a1);
-            }
-            const int g = wgi * HW + hh;
-            s[hh] = valid ? (a0 + a1) + (fb[2 * g] + fb[2 * g + 1]) : -INFINITY;
+          for (int cc = 0; cc < KP / 8; ++cc) {
+            const uint32_t L = row * row_bytes + (c0 + cc) * 16;
+            const uint4 w = *reinterpret_cast<const uint4*>(
+                bx + (L ^ (((L >> 7) & (uint32_t)p.kswz_mask) << 4)));
+            const float* fr = &f[cc * 8];
+            a0 = fmaf(bf_lo(w.x), fr[0], a0);
+            a1 = fmaf(bf_hi(w.x), fr[1], a1);
+            a0 = fmaf(bf_lo(w.y), fr[2], a0);
+            a1 = fmaf(bf_hi(w.y), fr[3], a1);
+            a0 = fmaf(bf_lo(w.z), fr[4], a0);
+            a1 = fmaf(bf_hi(w.z), fr[5], a1);
+            a0 = fmaf(bf_lo(w.w), fr[6], a0);
+            a1 = fmaf(bf_hi(w.w), fr[7], a1);
           }
+          sc = valid ? (a0 + a1) + (fb[0] + fb[1]) : -INFINITY;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_k[stage]);
-        if (epi_barrier_or(!ok)) {
+        if (epi_barrier_or_n<kEpiThreadsF>(!ok)) {
           aborted = true;
           break;
         }
-        // ---- softmax weights against the item's reference maximum (taken on the
-        // item's first tile; a later tile takes a new one only when a score exceeds it
-        // by more than 2^kRescaleLog2), per head, within the owning warpgroup
-        int over = 0;
-#pragma unroll
-        for (int hh = 0; hh < HW; ++hh) over |= s[hh] > m_ref[hh] + kRescaleLog2;
+        // ---- softmax weights of head wgi against the item's reference maximum (taken
+        // on the item's first tile; a later tile takes a new one only when a score
+        // exceeds it by more than 2^kRescaleLog2)
+        float alpha = 1.f;
         bool rescale = false;
-        float alpha[HW];
-#pragma unroll
-        for (int hh = 0; hh < HW; ++hh) alpha[hh] = 1.f;
-        if (k == 0 || wg_barrier_or(2 + wgi, over)) {
-#pragma unroll
-          for (int hh = 0; hh < HW; ++hh) {
-            const float mx = warp_max_f(s[hh]);
-            if (lane == 0) red[(wgi * HW + hh) * 4 + sub] = mx;
-          }
+        if (k == 0 || wg_barrier_or(2 + wgi, sc > m_ref + kRescaleLog2)) {
+          const float mx = warp_max_f(sc);
+          if (lane == 0) red[wgi * 4 + sub] = mx;
           named_barrier(2 + wgi, 128);
-#pragma unroll
-          for (int hh = 0; hh < HW; ++hh) {
-            const int g = wgi * HW + hh;
-            const float mt =
-                fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
-            if (k == 0) {
-              m_ref[hh] = mt;
-            } else if (mt > m_ref[hh] + kRescaleLog2) {
-              alpha[hh] = exp2f(m_ref[hh] - mt);
-              m_ref[hh] = mt;
-              rescale = true;
-            }
+          const float mt =
+              fmaxf(fmaxf(red[wgi * 4], red[wgi * 4 + 1]), fmaxf(red[wgi * 4 + 2], red[wgi * 4 + 3]));
+          if (k == 0) {
+            m_ref = mt;
+          } else if (mt > m_ref + kRescaleLog2) {
+            alpha = exp2f(m_ref - mt);
+            m_ref = mt;
+            rescale = true;
           }
           named_barrier(2 + wgi, 128);   // every warp has read red before it is reused
         }
         const uint32_t pb = it & 1u;
         // the weights buffer is free once the V MMA of tile it - 2 has finished
-        ok = mbar_wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u, abort_flag);
+        ok = wait(&pempty[pb], ((it >> 1) & 1u) ^ 1u);
         if (rescale) {
-          // rare: rescale columns 2g, 2g + 1 of the V accumulator (every lane this
-          // warp owns) once the V MMA of the previous tile has finished
-          ok = ok && mbar_wait(&pempty[(it - 1) & 1u], ((it - 1) >> 1) & 1u, abort_flag);
+          // rare: rescale columns 2 wgi, 2 wgi + 1 of the V accumulator (every lane
+          // this warp owns) once the V MMA of the previous tile has finished
+          ok = ok && wait(&pempty[(it - 1) & 1u], ((it - 1) >> 1) & 1u);
           tc_fence_after();
-#pragma unroll
-          for (int hh = 0; hh < HW; ++hh) {
-            if (alpha[hh] != 1.f) {
-              const uint32_t ta = tmem_base + lane_addr + p.v_col0 + 2 * (wgi * HW + hh);
-              float v[2];
-              tmem_ld2(ta, v);
-              tmem_wait_ld();
-              tmem_st2(ta, v[0] * alpha[hh], v[1] * alpha[hh]);
-            }
-          }
+          const uint32_t ta = tmem_base + lane_addr + p.v_col0 + 2 * wgi;
+          float v[2];
+          tmem_ld2(ta, v);
+          tmem_wait_ld();
+          tmem_st2(ta, v[0] * alpha, v[1] * alpha);
           tmem_wait_st();
           tc_fence_before();
         }
@@ -2177,7 +2152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // rows past the context: zero them in the V stage, so that the V MMA takes
           // zero weights times zeros whatever the cache holds there
           const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
-          ok = ok && mbar_wait(&full_v[vs], vph, abort_flag);
+          ok = ok && wait(&full_v[vs], vph);
           if (!valid) {
             unsigned char* vrow = sm + p.stv_off + vs * p.stv_bytes + row * 128;
             for (int vb = 0; vb < p.nvb; ++vb)
@@ -2186,16 +2161,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4*>(vrow + vb * p.vbox_bytes + c * 16) = make_uint4(0, 0, 0, 0);
           }
         }
-#pragma unroll
-        for (int hh = 0; hh < HW; ++hh) {
-          const int g = wgi * HW + hh;
-          const float pj = valid ? exp2f(s[hh] - m_ref[hh]) : 0.f;
-          l_part[hh] = l_part[hh] * alpha[hh] + pj;
+        {
+          const float pj = valid ? exp2f(sc - m_ref) : 0.f;
+          l_part = l_part * alpha + pj;
           const __nv_bfloat16 hi = __float2bfloat16_rn(pj);
           const __nv_bfloat16 lo = __float2bfloat16_rn(pj - __bfloat162float(hi));
-          // weight rows 2g (hi) and 2g + 1 (lo): row group (2g) / 8, rows (2g) % 8 and + 1
-          unsigned char* pg = sm + p.p_off + pb * 4096u + ((2 * g) >> 3) * 2048 +
-                              (row >> 3) * 128 + ((2 * g) & 7) * 16 + (row & 7) * 2;
+          // weight rows 2 wgi (hi) and 2 wgi + 1 (lo) of row group 0
+          unsigned char* pg = sm + p.p_off + pb * 4096u + (row >> 3) * 128 + ((2 * wgi) & 7) * 16 +
+                              (row & 7) * 2;
           *reinterpret_cast<__nv_bfloat16*>(pg) = hi;
           *reinterpret_cast<__nv_bfloat16*>(pg + 16) = lo;
         }
@@ -2203,43 +2176,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&pfull[pb]);   // one arrival per epilogue warp
         if (!ok) *abort_flag = 1;
-        // two phase buffers: the tile after next goes into this tile's buffer (its
-        // last reader, this tile's F MMA, has completed)
-        if (p.ne == 2 && ec.valid) write_e();
+        // the tile ne ahead goes into this tile's phase buffer (its last reader, this
+        // tile's F MMA, has completed)
+        if (e_more) write_e();
       }
       if (aborted) break;
       // ---------------------------------------------------------- item finish
-      // this warpgroup's heads: l over the item (per warp into red), m
-#pragma unroll
-      for (int hh = 0; hh < HW; ++hh) {
-        const int g = wgi * HW + hh;
-        const float l = warp_sum_f(l_part[hh]);
-        if (lane == 0) red[g * 4 + sub] = l;
-        if (row == 0) misc[g] = m_ref[hh];
+      {
+        const float l = warp_sum_f(l_part);
+        if (lane == 0) red[wgi * 4 + sub] = l;
+        if (row == 0) misc[wgi] = m_ref;
       }
       bool okv = true;
       if (r.ntiles > 0) {
         const uint32_t last = it - 1;
-        okv = __all_sync(0xffffffffu, mbar_wait(&pempty[last & 1u], (last >> 1) & 1u, abort_flag));
+        okv = __all_sync(0xffffffffu, wait(&pempty[last & 1u], (last >> 1) & 1u));
         tc_fence_after();
       }
-      named_barrier(1, kEpiThreads);            // red, misc visible; olat free
-      // TMEM lane g r_v + m holds head g's latent dim m in columns 2g (hi), 2g + 1 (lo)
-      const int gl = row / p.r_v;               // head of this warp's lanes (r_v >= 32)
+      named_barrier(1, kEpiThreadsF);           // red, misc visible; olat free
+      // TMEM lane g r_v + m (r_v = 32: sub-partition g) holds head g's latent dim m in
+      // columns 2g (hi) and 2g + 1 (lo)
       if (wgi == 0) {
         float v[2] = {0.f, 0.f};
         if (r.ntiles > 0 && okv) {
-          tmem_ld2(tmem_base + lane_addr + p.v_col0 + 2 * gl, v);
+          tmem_ld2(tmem_base + lane_addr + p.v_col0 + 2 * sub, v);
           tmem_wait_ld();
         }
         olat[row] = v[0] + v[1];
       }
       tc_fence_before();
-      named_barrier(1, kEpiThreads);            // olat complete
+      named_barrier(1, kEpiThreadsF);           // olat complete
       if constexpr (FUSE) {
         // One split per group: o = (W_up,v o_lat a + mu_v l a + v_self b) / (l a + b),
         // a = 2^(m - M), b = 2^(s_self - M), M = max(m, s_self) (base-2 scores).
-        for (int o = et; o < G * p.d; o += kEpiThreads) {
+        for (int o = et; o < G * p.d; o += kEpiThreadsF) {
           const int g = o / p.d, dd = o - g * p.d;
           const int h = r.hg * G + g;
           const size_t bh = (size_t)r.b * p.H + h;
@@ -2253,7 +2223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float* Wt = p.wupv_t + (size_t)h * p.d * p.r_v + dd;
           const float* ol = olat + g * p.r_v;
           float y0 = 0.f, y1 = 0.f;
-          for (int m0 = 0; m0 < p.r_v; m0 += 16) {
+#pragma unroll
+          for (int m0 = 0; m0 < 32; m0 += 16) {
             float wv[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) wv[e] = __ldg(Wt + (size_t)(m0 + e) * p.d);
@@ -2268,7 +2239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // split partials (m, l, sum p c_v) of the group's heads for decode_combine_kernel
-        for (int idx = et; idx < G * (2 + p.r_v); idx += kEpiThreads) {
+        for (int idx = et; idx < G * (2 + p.r_v); idx += kEpiThreadsF) {
           const int g = idx / (2 + p.r_v), m = idx - g * (2 + p.r_v);
           const size_t bh = (size_t)r.b * p.H + r.hg * G + g;
           float v;
@@ -2283,7 +2254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.partials[(bh * p.S + r.s) * (2 + p.r_v) + m] = v;
         }
       }
-      named_barrier(1, kEpiThreads);            // scratch free for the next item
+      named_barrier(1, kEpiThreadsF);           // scratch free for the next item
     }
   }
 
@@ -2505,16 +2476,16 @@ uint32_t tcf_layout(TcParams& p, int D, int G, int nst, int nst_v, int nbuf_b, i
 }
 
 // Whether the phase-operand kernel takes the shape: per head, RoPE over the whole
-// head of width 64 or 128, r_k of 16 or 32, and G = 128 / r_v of 2 or 4 heads per
-// item dividing H.  LLA_TC_FORM=u keeps such shapes on decode_tc_kernel.
+// head of width 64 or 128, r_k of 16 or 32, r_v = 32 (so the G = 4 heads of an item
+// fill the 128 rows of the transposed V MMA) and H a multiple of 4.  LLA_TC_FORM=u
+// keeps such shapes on decode_tc_kernel.
 bool tcf_shape(const lla_cfg& c) {
   const char* v = std::getenv("LLA_TC_FORM");
   if (v && v[0] == 'u') return false;
   if (c.mode != LLA_MODE_PER_HEAD || has_nope(c)) return false;
   if (c.d_head != 64 && c.d_head != 128) return false;
   if (c.r_k != 16 && c.r_k != 32) return false;
-  if (c.r_v != 32 && c.r_v != 64) return false;
-  return c.H % (128 / c.r_v) == 0;
+  return c.r_v == 32 && c.H % kGF == 0;
 }
 
 TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
@@ -2535,7 +2506,7 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
     // phase-operand kernel: three F buffers (3 n_f + 16 TMEM columns), then the most
     // latent bytes in flight with two phase buffers and one image buffer (both can be
     // forced: LLA_TCF_NE, LLA_TCF_NBUF)
-    const int G = 128 / c.r_v;
+    const int G = kGF;
     const int ne_f = env_int("LLA_TCF_NE", 0), nbuf_f = env_int("LLA_TCF_NBUF", 0);
     for (int ne : {2, 1}) {
       if (best_g || (ne_f && ne != ne_f)) continue;
@@ -2742,18 +2713,18 @@ cudaError_t launch_tc_nope(int G, bool shared, const CUtensorMap& mk, const CUte
   }
 }
 
-template <int D, int G, int KP>
+template <int D, int KP>
 cudaError_t launch_tcf_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
                          uint32_t smem, int grid, cudaStream_t s) {
   void (*kern)(CUtensorMap, CUtensorMap, TcParams) =
-      p.fuse_combine ? decode_tcf_kernel<D, G, KP, true> : decode_tcf_kernel<D, G, KP, false>;
+      p.fuse_combine ? decode_tcf_kernel<D, KP, true> : decode_tcf_kernel<D, KP, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch after the prep kernel: the producers wait for its
   // grid only before the first operand-image load
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kThreadsF);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -2764,19 +2735,12 @@ cudaError_t launch_tcf_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcP
   return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
 }
 
-cudaError_t launch_tcf(int D, int G, int KP, const CUtensorMap& mk, const CUtensorMap& mv,
+cudaError_t launch_tcf(int D, int KP, const CUtensorMap& mk, const CUtensorMap& mv,
                        const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
-#define LLA_TCF(DD, GG, KK) \
-  if (D == DD && G == GG && KP == KK) return launch_tcf_t<DD, GG, KK>(mk, mv, p, smem, grid, s)
-  LLA_TCF(128, 4, 16);
-  LLA_TCF(128, 4, 32);
-  LLA_TCF(128, 2, 16);
-  LLA_TCF(128, 2, 32);
-  LLA_TCF(64, 4, 16);
-  LLA_TCF(64, 4, 32);
-  LLA_TCF(64, 2, 16);
-  LLA_TCF(64, 2, 32);
-#undef LLA_TCF
+  if (D == 128 && KP == 16) return launch_tcf_t<128, 16>(mk, mv, p, smem, grid, s);
+  if (D == 128 && KP == 32) return launch_tcf_t<128, 32>(mk, mv, p, smem, grid, s);
+  if (D == 64 && KP == 16) return launch_tcf_t<64, 16>(mk, mv, p, smem, grid, s);
+  if (D == 64 && KP == 32) return launch_tcf_t<64, 32>(mk, mv, p, smem, grid, s);
   return cudaErrorNotSupported;
 }
 
@@ -2921,7 +2885,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
     cudaError_t pe = launch_prep_f(a, p, pl.G, s);
     if (pe != cudaSuccess) return pe;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    cudaError_t e = launch_tcf(a.d, pl.G, a.r_k, mk, mv, p, smem, grid, s);
+    cudaError_t e = launch_tcf(a.d, a.r_k, mk, mv, p, smem, grid, s);
     if (e == cudaSuccess && !p.fuse_combine) e = launch_combine(a, s);
     return e;
   }

@@ -165,9 +165,9 @@ def test_forced_split_count_is_clamped(monkeypatch):
 
 
 def test_phase_operand_kernel_workspace():
-    """Per-head shapes with r_k in {16, 32} and G = 128 / r_v heads per item run on
-    the phase-operand kernel, whose operand images are one [G r_k + 16, d] bf16 image
-    per (sequence, head group); LLA_TC_FORM=u keeps them on the per-head kernel, whose
+    """Per-head shapes with r_k in {16, 32} and r_v = 32 run on the phase-operand
+    kernel, whose operand images are one [4 r_k + 16, d] bf16 image per (sequence,
+    group of four heads); LLA_TC_FORM=u keeps them on the per-head kernel, whose
     images are per (sequence, head)."""
     import os
     cfg = lla.Cfg(4, 16, 128, 16, 32)
