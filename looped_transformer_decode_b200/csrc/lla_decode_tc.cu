@@ -2009,10 +2009,18 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 #pragma unroll
     for (int q = 0; q < WG_PAIRS; ++q) ef[q] = make_float2(1.f, 0.f);
     uint32_t ie = 0;   // phase tiles written
-    // This thread's row of the next phase tile into buffer ie % ne: entries
-    // (2i, 2i + 1) = (cos, -sin) of pair i, 128-byte swizzled K-major rows.
-    auto write_e = [&]() {
+    // The factors of the next phase tile (its position was loaded a tile ago), and the
+    // position of the one after it.
+    auto advance_e = [&]() {
       advance_rope(pos_pref);
+      e_more = ec.valid;
+      pos_pref = cursor_pos(p, ec, row);      // used by the next advance
+      cursor_next(p, ctx_s, ec);
+    };
+    // This thread's row of that tile into buffer ie % ne: entries (2i, 2i + 1) =
+    // (cos, -sin) of pair i, 128-byte swizzled K-major rows.  The caller fences and
+    // arrives on efull[(ie - 1) % ne].
+    auto store_e = [&]() {
       unsigned char* eb = sm + p.e_off + (ie % p.ne) * p.e_bytes;
 #pragma unroll
       for (int c = 0; c < WG_PAIRS / 4; ++c) {
@@ -2029,15 +2037,15 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         memcpy(&v.w, &b3, 4);
         *reinterpret_cast<uint4*>(eb + blk * (kTile * 128) + row * 128 + ((ch ^ (row & 7)) << 4)) = v;
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&efull[ie % p.ne]);
-      e_more = ec.valid;
-      pos_pref = cursor_pos(p, ec, row);      // used by the next call
-      cursor_next(p, ctx_s, ec);
       ++ie;
     };
-    for (int k = 0; k < p.ne && e_more; ++k) write_e();
+    for (int k = 0; k < p.ne && e_more; ++k) {
+      advance_e();
+      store_e();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&efull[(ie - 1) % p.ne]);
+    }
 
     uint32_t it = 0;
     bool aborted = false;
@@ -2077,6 +2085,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[acc]);
+        // the phase tile ne ahead: its factors now (arithmetic that overlaps the
+        // waits below), its rows with this tile's weights
+        const bool e_now = e_more;
+        if (e_now) advance_e();
 
         // s = sum_m c_m F_m + F_M for head wgi, with this token row's latents read
         // from the swizzled K tile
@@ -2108,16 +2120,20 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_k[stage]);
-        if (epi_barrier_or_n<kEpiThreadsF>(!ok)) {
-          aborted = true;
-          break;
-        }
         // ---- softmax weights of head wgi against the item's reference maximum (taken
         // on the item's first tile; a later tile takes a new one only when a score
-        // exceeds it by more than 2^kRescaleLog2)
+        // exceeds it by more than 2^kRescaleLog2).  One barrier of the warpgroup asks
+        // whether any thread needs more than the common case: the first tile, a new
+        // maximum, or a failed wait.  A warpgroup that saw a wait fail leaves the tile
+        // loop; the others then find their next hand-off unanswered, time out and
+        // follow, and all warpgroups agree once more before the item's finish.
         float alpha = 1.f;
         bool rescale = false;
-        if (k == 0 || wg_barrier_or(2 + wgi, sc > m_ref + kRescaleLog2)) {
+        if (wg_barrier_or(2 + wgi, k == 0 || !ok || sc > m_ref + kRescaleLog2)) {
+          if (wg_barrier_or(2 + wgi, !ok)) {
+            aborted = true;
+            break;
+          }
           const float mx = warp_max_f(sc);
           if (lane == 0) red[wgi * 4 + sub] = mx;
           named_barrier(2 + wgi, 128);
@@ -2172,15 +2188,18 @@ __global__ void __launch_bounds__(kThreadsF, 1)
           *reinterpret_cast<__nv_bfloat16*>(pg) = hi;
           *reinterpret_cast<__nv_bfloat16*>(pg + 16) = lo;
         }
+        // the phase tile ne ahead goes into this tile's buffer (its last reader, this
+        // tile's F MMA, has completed); one proxy fence covers both writes
+        if (e_now) store_e();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&pfull[pb]);   // one arrival per epilogue warp
+        if (lane == 0) {
+          mbar_arrive(&pfull[pb]);               // one arrival per epilogue warp
+          if (e_now) mbar_arrive(&efull[(ie - 1) % p.ne]);
+        }
         if (!ok) *abort_flag = 1;
-        // the tile ne ahead goes into this tile's phase buffer (its last reader, this
-        // tile's F MMA, has completed)
-        if (e_more) write_e();
       }
-      if (aborted) break;
+      if (epi_barrier_or_n<kEpiThreadsF>(aborted)) break;
       // ---------------------------------------------------------- item finish
       {
         const float l = warp_sum_f(l_part);
