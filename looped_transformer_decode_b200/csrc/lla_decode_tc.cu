@@ -1641,6 +1641,18 @@ __global__ void __launch_bounds__(kThreads2, 1)
 // heads at once, D_v^T[G r_v x 2G] += C_v^T P^T, of which only the diagonal blocks
 // are read (as in the LLA-2D kernel).  Both are exact reorderings of the same sums.
 
+// Slot of a ring of n entries and the parity of its current pass, stepped by one
+// (no division per step).
+struct RingPos {
+  uint32_t slot = 0, phase = 0;
+  __device__ __forceinline__ void next(uint32_t n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 // Operand image of one item (sequence b, group of G heads) for decode_tcf_kernel:
 // [n_f rows x d] bf16 in the 128-byte-swizzled K-major layout (d / 64 column blocks
 // of n_f x 128 bytes; 16-byte chunk c of row n at chunk c ^ (n % 8)).  Row g r_k + m
@@ -1735,6 +1747,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
   constexpr int G = kGF;
   constexpr int WG_PAIRS = D / 2 / kEpiWGF;  // RoPE pairs of a token row each warpgroup writes
+  constexpr uint32_t NACC = 3;               // F buffers in TMEM
+  constexpr int BOXK = 64;                   // K latent boxes: 64 columns, 128-byte swizzled rows
   static_assert(WG_PAIRS % 4 == 0 && KP % 16 == 0, "shape");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -1827,6 +1841,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       uint64_t* fullb = kside ? full_k : full_v;
       uint64_t* emptyb = kside ? empty_k : empty_v;
       uint32_t it = 0, jn = 0;
+      RingPos rs;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
@@ -1843,8 +1858,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                     p.b_img_bytes, &bfull[buf]);
           ++jn;
         }
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
-          const uint32_t stage = it % nst, ph = (it / nst) & 1u;
+        for (int k = 0; k < r.ntiles; ++k, ++it, rs.next(nst)) {
+          const uint32_t stage = rs.slot, ph = rs.phase;
           if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {   // producers suspend
             ok = false;
             break;
@@ -1855,7 +1870,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             unsigned char* st = sm + p.st_off + stage * p.st_bytes;
             for (int kb = 0; kb < p.nkb; ++kb)
               tma_load_3d(st + kb * p.box_bytes, map, &fullb[stage],
-                          r.hg * (G * KP) + kb * p.box_k, y, r.b);
+                          r.hg * (G * KP) + kb * BOXK, y, r.b);
           } else {
             mbar_arrive_expect_tx(&fullb[stage], p.tx_v);
             unsigned char* st = sm + p.stv_off + stage * p.stv_bytes;
@@ -1893,6 +1908,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       const uint32_t e_base = smem_addr(sm + p.e_off);
       const uint32_t b_base0 = smem_addr(sm + p.b_off);
       uint32_t it = 0, jn = 0;
+      RingPos ra;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
@@ -1901,9 +1917,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         if (!wait(&bfull[buf], bph)) break;
         ++jn;
         const uint32_t b_base = b_base0 + buf * p.b_head_bytes;
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
-          const uint32_t e = it % p.ne, eph = (it / p.ne) & 1u;
-          const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+        for (int k = 0; k < r.ntiles; ++k, ++it, ra.next(NACC)) {
+          const uint32_t e = it & 1u, eph = (it >> 1) & 1u;     // two phase buffers
+          const uint32_t acc = ra.slot, aph = ra.phase;
           if (!wait(&efull[e], eph) || !wait(&tempty[acc], aph ^ 1u)) {
             ok = false;
             break;
@@ -1934,12 +1950,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       const uint32_t sbo_v = 16u * p.cvb;
       const uint32_t p_base = smem_addr(sm + p.p_off);
       uint32_t it = 0;
+      RingPos rv;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
+        for (int k = 0; k < r.ntiles; ++k, ++it, rv.next(p.nst_v)) {
           const uint32_t pb = it & 1u;
-          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          const uint32_t vs = rv.slot, vph = rv.phase;
           if (!wait(&pfull[pb], (it >> 1) & 1u) || !wait(&full_v[vs], vph)) {
             ok = false;
             break;
@@ -2021,7 +2038,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     // (cos, -sin) of pair i, 128-byte swizzled K-major rows.  The caller fences and
     // arrives on efull[(ie - 1) % ne].
     auto store_e = [&]() {
-      unsigned char* eb = sm + p.e_off + (ie % p.ne) * p.e_bytes;
+      unsigned char* eb = sm + p.e_off + (ie & 1u) * p.e_bytes;
 #pragma unroll
       for (int c = 0; c < WG_PAIRS / 4; ++c) {
         const int pair0 = wgi * WG_PAIRS + c * 4;
@@ -2039,15 +2056,16 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       }
       ++ie;
     };
-    for (int k = 0; k < p.ne && e_more; ++k) {
+    for (int k = 0; k < 2 && e_more; ++k) {
       advance_e();
       store_e();
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&efull[(ie - 1) % p.ne]);
+      if (lane == 0) mbar_arrive(&efull[(ie - 1) & 1u]);
     }
 
     uint32_t it = 0;
+    RingPos ra, rk;                           // F buffers, K stages
     bool aborted = false;
     for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
       const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
@@ -2064,9 +2082,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int off = row * 128; off < p.d * p.r_v * 4; off += 128 * 128)
           asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wrow + off));
       }
-      for (int k = 0; k < r.ntiles; ++k, ++it) {
-        const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
-        const uint32_t stage = it % p.nst, kph = (it / p.nst) & 1u;
+      for (int k = 0; k < r.ntiles; ++k, ++it, ra.next(NACC), rk.next(p.nst)) {
+        const uint32_t acc = ra.slot, aph = ra.phase;
+        const uint32_t stage = rk.slot, kph = rk.phase;
         const int t0 = r.tok0 + k * kTile;
         const int cnt = min(kTile, r.tok_end - t0);
         const bool valid = row < cnt;
@@ -2096,16 +2114,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         float sc;
         {
           const unsigned char* st = sm + p.st_off + stage * p.st_bytes;
-          const uint32_t row_bytes = (uint32_t)p.box_k * 2;
           const int e0 = wgi * KP;                         // first latent column of the head
-          const unsigned char* bx = st + (e0 / p.box_k) * p.box_bytes;
-          const uint32_t c0 = (uint32_t)(e0 % p.box_k) * 2 / 16;
+          const unsigned char* bx = st + (e0 / BOXK) * (kTile * BOXK * 2) + row * (BOXK * 2);
+          const uint32_t c0 = (uint32_t)(e0 % BOXK) / 8;   // its first 16-byte chunk
           float a0 = 0.f, a1 = 0.f;
 #pragma unroll
           for (int cc = 0; cc < KP / 8; ++cc) {
-            const uint32_t L = row * row_bytes + (c0 + cc) * 16;
-            const uint4 w = *reinterpret_cast<const uint4*>(
-                bx + (L ^ (((L >> 7) & (uint32_t)p.kswz_mask) << 4)));
+            const uint4 w = *reinterpret_cast<const uint4*>(bx + (((c0 + cc) ^ (row & 7)) << 4));
             const float* fr = &f[cc * 8];
             a0 = fmaf(bf_lo(w.x), fr[0], a0);
             a1 = fmaf(bf_hi(w.x), fr[1], a1);
@@ -2167,7 +2182,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         if (cnt < kTile && wgi == 0) {
           // rows past the context: zero them in the V stage, so that the V MMA takes
           // zero weights times zeros whatever the cache holds there
-          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;   // partial tiles only
           ok = ok && wait(&full_v[vs], vph);
           if (!valid) {
             unsigned char* vrow = sm + p.stv_off + vs * p.stv_bytes + row * 128;
@@ -2195,7 +2210,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&pfull[pb]);               // one arrival per epilogue warp
-          if (e_now) mbar_arrive(&efull[(ie - 1) % p.ne]);
+          if (e_now) mbar_arrive(&efull[(ie - 1) & 1u]);
         }
         if (!ok) *abort_flag = 1;
       }
@@ -2522,13 +2537,13 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   // buffers when they fit.
   int best_g = 0, best_nst = 0, best_nst_v = 0, best_nacc = 1;
   if (tcf_shape(c)) {
-    // phase-operand kernel: three F buffers (3 n_f + 16 TMEM columns), then the most
-    // latent bytes in flight with two phase buffers and one image buffer (both can be
-    // forced: LLA_TCF_NE, LLA_TCF_NBUF)
+    // phase-operand kernel: three F buffers (3 n_f + 16 TMEM columns), two phase
+    // buffers, then the most latent bytes in flight with one image buffer
+    // (LLA_TCF_NBUF=2 forces two)
     const int G = kGF;
-    const int ne_f = env_int("LLA_TCF_NE", 0), nbuf_f = env_int("LLA_TCF_NBUF", 0);
-    for (int ne : {2, 1}) {
-      if (best_g || (ne_f && ne != ne_f)) continue;
+    const int nbuf_f = env_int("LLA_TCF_NBUF", 0);
+    for (int ne : {2}) {
+      if (best_g) continue;
       for (int nbuf : {1, 2}) {
         if (best_g || (nbuf_f && nbuf != nbuf_f) || (!nbuf_f && nbuf == 2)) continue;
         TcParams p{};
