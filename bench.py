@@ -64,6 +64,10 @@ def parse():
                    help="measure the default workload only (no sub-records of the others)")
     p.add_argument("--encode-tokens", type=int, default=0,
                    help="override the workload's tokens encoded per step (profiling aid)")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's batch (profiling aid: a smaller capture)")
+    p.add_argument("--layers", type=int, default=0,
+                   help="override the workload's layer count (profiling aid)")
     p.add_argument("--path", default="latent", choices=["latent", "full"],
                    help="latent: decode over the latent cache (rebuild on read); full: the "
                         "full-memory fast path (K/V rebuilt once per token into a full bf16 "
@@ -598,7 +602,7 @@ def measure(lla, w, args, device, world, rank, local, dist_on, steps, warmup, pa
     enc_gbs = append_bytes / (enc_avg * 1e-3) / 1e9
     traffic_table = NCU_TRAFFIC_FULL if full else NCU_TRAFFIC
     traffic = ((NCU_TRAFFIC_DECOUPLED.get((w.name, d_rope)) if d_rope else traffic_table.get(w.name))
-               if not (args.encode_tokens or evict_arg) else None)
+               if not (args.encode_tokens or evict_arg or args.batch) else None)
     dkname = ("lla_full_decode_attn (full_decode_kernel [+ combine])" if full
               else "lla_decode_attn (prep + partial kernel [+ combine])")
     dec_roof = {"bound": "hbm", "kernel": dkname, "achieved": round(dec_gbs, 1), "peak": peak,
@@ -704,6 +708,11 @@ def run_gpu(args):
     w = synth.WORKLOADS[args.workload]
     if args.encode_tokens:
         w = dataclasses.replace(w, encode_tokens=args.encode_tokens)
+    if args.batch:
+        w = dataclasses.replace(w, B=args.batch, encode_tokens=min(w.encode_tokens, args.batch)
+                                if w.encode_tokens <= w.B else w.encode_tokens)
+    if args.layers:
+        w = dataclasses.replace(w, layers=args.layers)
     rec = measure(lla, w, args, device, world, rank, local, dist_on, args.steps, args.warmup,
                   path=args.path, d_rope=args.d_rope, evict_arg=args.evict, eager=args.eager,
                   with_e2e=not args.no_e2e)
@@ -718,7 +727,7 @@ def run_gpu(args):
     if args.path == "full":
         line["e2e_note"] = "no end-to-end line on the full-memory path"
     if not args.no_sub and args.workload == DEFAULT_WORKLOAD and args.path == "latent" \
-            and not (args.d_rope or args.evict or args.encode_tokens):
+            and not (args.d_rope or args.evict or args.encode_tokens or args.batch or args.layers):
         subs = []
         for name in SUB_WORKLOADS:
             sw = synth.WORKLOADS[name]
