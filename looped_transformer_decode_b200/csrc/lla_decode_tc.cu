@@ -228,6 +228,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Slot of a ring of n entries and the parity of its current pass, stepped by one
+// (no division per step).
+struct RingPos {
+  uint32_t slot = 0, phase = 0;
+  __device__ __forceinline__ void next(uint32_t n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 struct ItemRange {
   int b, hg, s, tok0, tok_end, ntiles;
 };
@@ -629,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* fullb = kside ? full_k : full_v;
       uint64_t* emptyb = kside ? empty_k : empty_v;
       uint32_t it = 0, jn = 0;
+      RingPos rs;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
@@ -647,8 +660,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     p.ops_bias + head0 * p.bias_head_bytes, G * p.bias_head_bytes, &bfull[buf]);
           ++jn;
         }
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
-          const uint32_t stage = it % nst, ph = (it / nst) & 1u;
+        for (int k = 0; k < r.ntiles; ++k, ++it, rs.next(nst)) {
+          const uint32_t stage = rs.slot, ph = rs.phase;
           if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -703,6 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sbo_a = 16u * p.box_k;
       const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 0, 0);   // rows alias
       uint32_t it = 0, jn = 0;
+      RingPos rk, ra;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
@@ -715,9 +729,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++jn;
         const uint32_t b_base = smem_addr(sm + p.b_off + buf * G * ops_head_bytes);
         const uint32_t bias_base = smem_addr(sm + p.bias_off + buf * G * p.bias_head_bytes);
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
-          const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
-          const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+        for (int k = 0; k < r.ntiles; ++k, ++it, rk.next(p.nst), ra.next(p.nacc)) {
+          const uint32_t stage = rk.slot, ph = rk.phase;
+          const uint32_t acc = ra.slot, aph = ra.phase;
           if (!mbar_wait(&full_k[stage], ph, abort_flag) ||
               !mbar_wait(&tempty[acc], aph ^ 1u, abort_flag)) {
             ok = false;
@@ -756,12 +770,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sbo_v = 16u * p.cvb;          // 8 token rows of one MN box
       const uint32_t p_base = smem_addr(sm + p.p_off);
       uint32_t it = 0;
+      RingPos rv;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
+        for (int k = 0; k < r.ntiles; ++k, ++it, rv.next(p.nst_v)) {
           const uint32_t pb = it & 1u;
-          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          const uint32_t vs = rv.slot, vph = rv.phase;
           if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag) ||
               !mbar_wait(&full_v[vs], vph, abort_flag)) {
             ok = false;
@@ -837,6 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cursor_next(p, ctx_s, pc);
 
     uint32_t it = 0;
+    RingPos ra;
     bool aborted = false;
     for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
       const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
@@ -864,8 +880,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(wrow + off));
         }
       }
-      for (int k = 0; k < r.ntiles; ++k, ++it) {
-        const uint32_t acc = it % p.nacc, aph = (it / p.nacc) & 1u;
+      for (int k = 0; k < r.ntiles; ++k, ++it, ra.next(p.nacc)) {
+        const uint32_t acc = ra.slot, aph = ra.phase;
         const int t0 = r.tok0 + k * kTile;
         const int cnt = min(kTile, r.tok_end - t0);
         const bool valid = row < cnt;
@@ -1258,6 +1274,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       uint64_t* fullb = kside ? full_k : full_v;
       uint64_t* emptyb = kside ? empty_k : empty_v;
       uint32_t it = 0, jn = 0;
+      RingPos rs;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
@@ -1273,8 +1290,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
                     p.ops_bias + head0 * p.bias_head_bytes, HP * p.bias_head_bytes, &bfull[buf]);
           ++jn;
         }
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
-          const uint32_t stage = it % nst, ph = (it / nst) & 1u;
+        for (int k = 0; k < r.ntiles; ++k, ++it, rs.next(nst)) {
+          const uint32_t stage = rs.slot, ph = rs.phase;
           if (!mbar_wait(&emptyb[stage], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -1317,7 +1334,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(128, NS);
       const uint32_t sbo_a = 16u * p.box_k;
       const uint64_t odesc = smem_desc(smem_addr(sm + p.ones_off), 128, 0, 0);   // rows alias
-      uint32_t it = 0, jn = 0, u = 0;
+      uint32_t it = 0, jn = 0;
+      RingPos rk, ra;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
@@ -1330,16 +1348,16 @@ __global__ void __launch_bounds__(kThreads2, 1)
         ++jn;
         const uint32_t b_base = smem_addr(sm + p.b_off + buf * HP * ops_head_bytes);
         const uint32_t bias_base = smem_addr(sm + p.bias_off + buf * HP * p.bias_head_bytes);
-        for (int k = 0; ok && k < r.ntiles; ++k, ++it) {
-          const uint32_t stage = it % p.nst, ph = (it / p.nst) & 1u;
+        for (int k = 0; ok && k < r.ntiles; ++k, ++it, rk.next(p.nst)) {
+          const uint32_t stage = rk.slot, ph = rk.phase;
           if (!mbar_wait(&full_k[stage], ph, abort_flag)) {
             ok = false;
             break;
           }
           const uint32_t st_addr = smem_addr(sm + p.st_off + stage * p.st_bytes);
 #pragma unroll 1
-          for (int g = 0; g < HP; ++g, ++u) {
-            const uint32_t acc = u % p.nacc, aph = (u / p.nacc) & 1u;
+          for (int g = 0; g < HP; ++g, ra.next(p.nacc)) {
+            const uint32_t acc = ra.slot, aph = ra.phase;
             if (!(p.poll ? mbar_wait_poll(&tempty[acc], aph ^ 1u, abort_flag)
                          : mbar_wait(&tempty[acc], aph ^ 1u, abort_flag))) {
               ok = false;
@@ -1377,12 +1395,13 @@ __global__ void __launch_bounds__(kThreads2, 1)
       const uint32_t boxes_per_block = 128u / p.cvb;
       const uint32_t p_base = smem_addr(sm + p.p_off);
       uint32_t it = 0;
+      RingPos rv;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const ItemRange r = item_range(p, ctx_s, item, false);
-        for (int k = 0; k < r.ntiles; ++k, ++it) {
+        for (int k = 0; k < r.ntiles; ++k, ++it, rv.next(p.nst_v)) {
           const uint32_t pb = it & 1u;
-          const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;
+          const uint32_t vs = rv.slot, vph = rv.phase;
           if (!mbar_wait(&pfull[pb], (it >> 1) & 1u, abort_flag) ||
               !mbar_wait(&full_v[vs], vph, abort_flag)) {
             ok = false;
@@ -1454,7 +1473,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
     int pos_next = cursor_pos(p, pc, row);
     cursor_next(p, ctx_s, pc);
 
-    uint32_t it = 0, u = 0;
+    uint32_t it = 0;
+    RingPos ra;
     bool aborted = false;
     for (int item = blockIdx.x; !aborted && item < p.n_items; item += gridDim.x) {
       const ItemRange r = item_range(p, ctx_s, item, et == 0 && !ctx_s);
@@ -1466,8 +1486,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
         const uint32_t par = it & 1u;
         bool ok = true;
 #pragma unroll 1
-        for (int g = 0; g < HP; ++g, ++u) {
-          const uint32_t acc = u % p.nacc, aph = (u / p.nacc) & 1u;
+        for (int g = 0; g < HP; ++g, ra.next(p.nacc)) {
+          const uint32_t acc = ra.slot, aph = ra.phase;
           ok = ok && (p.poll ? mbar_wait_poll(&tfull[acc], aph, abort_flag)
                              : mbar_wait(&tfull[acc], aph, abort_flag));
           tc_fence_after();
@@ -1640,18 +1660,6 @@ __global__ void __launch_bounds__(kThreads2, 1)
 // latents instead of d/2 complex products.  The V sum is taken transposed for the G
 // heads at once, D_v^T[G r_v x 2G] += C_v^T P^T, of which only the diagonal blocks
 // are read (as in the LLA-2D kernel).  Both are exact reorderings of the same sums.
-
-// Slot of a ring of n entries and the parity of its current pass, stepped by one
-// (no division per step).
-struct RingPos {
-  uint32_t slot = 0, phase = 0;
-  __device__ __forceinline__ void next(uint32_t n) {
-    if (++slot == n) {
-      slot = 0;
-      phase ^= 1u;
-    }
-  }
-};
 
 // Operand image of one item (sequence b, group of G heads) for decode_tcf_kernel:
 // [n_f rows x d] bf16 in the 128-byte-swizzled K-major layout (d / 64 column blocks
