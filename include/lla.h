@@ -211,7 +211,8 @@ size_t lla_decode_workspace_bytes(const lla_cfg* cfg, int32_t B, int32_t n_cap);
  *   positions     device int32 [B][n_cap]: position of each history token
  *   q_pos         device int32 [B]: position of the in-flight token
  *   c_k, c_v      device bf16 latent caches: per head [B][n_cap][H][r_k] / [..][r_v];
- *                 LLA-2D [B][n_cap][r_k] / [B][n_cap][r_v]
+ *                 LLA-2D [B][n_cap][r_k] / [B][n_cap][r_v].  Rows at or past ctx_len[b]
+ *                 never reach the output, whatever they hold (NaN included).
  *   out           device fp32 [B][H][d]
  *   ws            device workspace of >= lla_decode_workspace_bytes(cfg, B, n_cap)
  * Work is launched on `stream` only; there is no host synchronisation.

@@ -988,6 +988,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
           }
+          if (cnt < kTile) {
+            // rows past the context: zero them in the V stage, so that the V MMA takes
+            // zero weights times zeros whatever the cache holds there
+            const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;   // partial tiles only
+            ok = ok && mbar_wait(&full_v[vs], vph, abort_flag);
+            if (!valid) {
+              const uint32_t rbytes = (uint32_t)p.cvb * 2;                 // bytes of a box row
+              unsigned char* vrow = sm + p.stv_off + vs * p.stv_bytes + row * rbytes;
+              for (int bx = 0; bx < G * p.nvb; ++bx)
+                for (uint32_t c = 0; c < rbytes; c += 16)
+                  *reinterpret_cast<uint4*>(vrow + bx * p.vbox_bytes + c) = make_uint4(0, 0, 0, 0);
+            }
+          }
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float pj = valid ? exp2f(s[g] - m_ref[g]) : 0.f;
@@ -1561,6 +1574,19 @@ __global__ void __launch_bounds__(kThreads2, 1)
             }
             tmem_wait_st();
             tc_fence_before();
+          }
+          if (cnt < kTile && wgi == 0) {
+            // rows past the context: zero them in the loaded boxes of the V stage, so
+            // that the V MMA takes zero weights times zeros whatever the cache holds
+            const uint32_t vs = it % p.nst_v, vph = (it / p.nst_v) & 1u;   // partial tiles only
+            ok = ok && mbar_wait(&full_v[vs], vph, abort_flag);
+            if (!valid) {
+              const uint32_t rbytes = (uint32_t)p.cvb * 2;                 // bytes of a box row
+              unsigned char* vrow = sm + p.stv_off + vs * p.stv_bytes + row * rbytes;
+              for (int bx = 0; bx < p.nvb; ++bx)
+                for (uint32_t c = 0; c < rbytes; c += 16)
+                  *reinterpret_cast<uint4*>(vrow + bx * p.vbox_bytes + c) = make_uint4(0, 0, 0, 0);
+            }
           }
           const float pj = valid ? exp2f(sc - m_ref) : 0.f;
           l_part = l_part * alpha + pj;

@@ -235,6 +235,38 @@ def test_per_head_kernel_on_phase_operand_shapes(spec, monkeypatch):
     assert lla.decode_status(dev.ws) == 0
 
 
+NAN_TAIL = [
+    (O.Cfg(4, 2, 128, 96, 160), 2, 300, [300, 190], "tensor_core"),     # per-head kernel
+    (O.Cfg(4, 4, 128, 16, 32), 2, 300, [300, 190], "tensor_core"),      # phase-operand kernel
+    (O.Cfg(2, 4, 64, 32, 48, O.MODE_2D), 2, 300, [300, 150], "tensor_core"),   # LLA-2D kernel
+    (O.Cfg(4, 2, 64, 16, 32), 1, 2000, [1500], "tensor_core"),          # several splits
+    (O.Cfg(4, 2, 128, 96, 160), 2, 300, [300, 190], "cuda_core"),
+]
+
+
+@pytest.mark.parametrize("spec", NAN_TAIL, ids=lambda s: f"T{s[0].T}H{s[0].H}d{s[0].d}r{s[0].r_k}_{s[0].r_v}m{s[0].mode}n{s[2]}_{s[4]}")
+def test_cache_rows_past_the_context_are_never_used(spec, monkeypatch):
+    """Cache rows at or past ctx_len[b] may hold anything (here NaN): the output is
+    the oracle's over the first ctx_len rows.  The tensor-core kernels stream whole
+    128-token tiles, so they zero those rows of the staged V tile before the V MMA
+    (zero weights times NaN would be NaN), and mask their scores."""
+    cfg, B, n_cap, ctx, path = spec
+    if path == "cuda_core":
+        monkeypatch.setenv("LLA_DECODE_PATH", "cuda_core")
+    case = decode_case(cfg, B, n_cap, seed=700 + n_cap, ctx_len=ctx)
+    dev = DeviceCase(case)
+    nan = torch.tensor(float("nan"), dtype=torch.bfloat16, device="cuda")
+    for b, n in enumerate(case.ctx_len):
+        dev.c_k[b, int(n):] = nan
+        dev.c_v[b, int(n):] = nan
+    for t in (0, cfg.T - 1):
+        got = dev.decode(t)
+        assert np.isfinite(got).all(), t
+        err = rel_err(got, expected(case, t))
+        assert err.max() <= ATTN_TOL, (t, err.max())
+    assert lla.decode_status(dev.ws) == 0
+
+
 def test_decode_status_bits_for_bad_device_inputs():
     cfg = O.Cfg(4, 2, 64, 16, 32)
     case = decode_case(cfg, 2, 200, seed=9)
