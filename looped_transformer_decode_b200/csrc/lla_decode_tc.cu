@@ -71,6 +71,7 @@ struct TcParams {
   // LLA-2D kernel: B-operand buffers, P rows (N of the V MMA), 128-row blocks of r_v
   int nbuf_b, n_p, m_v;
   int poll;                                  // per-head hand-offs poll instead of suspending
+  uint32_t nap_ns, enap_ns;                  // naps between polls: MMA issuers, epilogue
   // fused split combine (per-head kernel): the CTA that finishes a group's last split
   // merges the splits, adds the in-flight token and up-projects with W_up,v
   const float* q;                            // [B][H][d]
@@ -1804,9 +1805,22 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
-  // hand-off waits: polled (the default, LLA_TC_POLL=1) or suspending
+  // Hand-off waits (LLA_TC_POLL): 2, the default, polls with a nap between polls,
+  // 1 polls, 0 suspends.  The kernel is bound by its instruction issue, and a warp
+  // spinning on a barrier takes issue slots from the epilogue warps of its
+  // sub-partition; napping gives them back at the cost of noticing the phase up to a
+  // nap late.  The MMA issuers, usually a tile or two ahead of the epilogue, nap
+  // longer (LLA_TC_NAP ns, 1000) than the epilogue (LLA_TC_ENAP ns, 64).  Measured on
+  // the 21.3x workload: 9.5% faster than polling, which was 1% faster than suspending.
   auto wait = [&](uint64_t* bar, uint32_t parity) {
-    return p.poll ? mbar_wait_poll(bar, parity, abort_flag) : mbar_wait(bar, parity, abort_flag);
+    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.enap_ns)
+           : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
+                       : mbar_wait(bar, parity, abort_flag);
+  };
+  auto wait_mma = [&](uint64_t* bar, uint32_t parity) {
+    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.nap_ns)
+           : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
+                       : mbar_wait(bar, parity, abort_flag);
   };
 
   if (threadIdx.x == 0) {
@@ -1948,13 +1962,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         const ItemRange r = item_range(p, ctx_s, item, false);
         if (r.ntiles == 0) continue;
         const uint32_t buf = jn % p.nbuf_b, bph = (jn / p.nbuf_b) & 1u;
-        if (!wait(&bfull[buf], bph)) break;
+        if (!wait_mma(&bfull[buf], bph)) break;
         ++jn;
         const uint32_t b_base = b_base0 + buf * p.b_head_bytes;
         for (int k = 0; k < r.ntiles; ++k, ++it, ra.next(NACC)) {
           const uint32_t e = it & 1u, eph = (it >> 1) & 1u;     // two phase buffers
           const uint32_t acc = ra.slot, aph = ra.phase;
-          if (!wait(&efull[e], eph) || !wait(&tempty[acc], aph ^ 1u)) {
+          if (!wait_mma(&efull[e], eph) || !wait_mma(&tempty[acc], aph ^ 1u)) {
             ok = false;
             break;
           }
@@ -1991,7 +2005,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int k = 0; k < r.ntiles; ++k, ++it, rv.next(p.nst_v)) {
           const uint32_t pb = it & 1u;
           const uint32_t vs = rv.slot, vph = rv.phase;
-          if (!wait(&pfull[pb], (it >> 1) & 1u) || !wait(&full_v[vs], vph)) {
+          if (!wait_mma(&pfull[pb], (it >> 1) & 1u) || !wait_mma(&full_v[vs], vph)) {
             ok = false;
             break;
           }
@@ -2940,7 +2954,9 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   const CUtensorMapSwizzle swz = p.box_k == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
-  p.poll = env_int("LLA_TC_POLL", 1);
+  p.poll = env_int("LLA_TC_POLL", 2);
+  p.nap_ns = (uint32_t)env_int("LLA_TC_NAP", 1000);
+  p.enap_ns = (uint32_t)env_int("LLA_TC_ENAP", 64);
   p.lat_hk = (int)a.lat_head_k;
   p.lat_hv = (int)a.lat_head_v;
   if (pl.fform) {

@@ -111,6 +111,26 @@ __device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity,
   }
 }
 
+// As mbar_wait_poll, but napping `nap_ns` between polls, so that a warp that waits
+// long takes few issue slots from the warps sharing its sub-partition while still
+// noticing the phase within about nap_ns.
+__device__ __forceinline__ bool mbar_wait_nap(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, uint32_t nap_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(nap_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ named barriers
 
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
