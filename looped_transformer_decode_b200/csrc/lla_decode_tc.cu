@@ -1805,11 +1805,11 @@ __global__ void __launch_bounds__(kThreadsF, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
-  // Hand-off waits (LLA_TC_POLL): 1, the default, polls; 2 polls with a nap between
-  // polls (the MMA issuers, usually a tile or two ahead of the epilogue, LLA_TC_NAP ns,
-  // 1000; the epilogue LLA_TC_ENAP ns, 64); 0 suspends.  Measured on the 21.3x
-  // workload: in graph-replayed steps polling is the fastest (537 against 561 us with
-  // naps); single calls after an L2 flush were faster with naps on some boxes.
+  // Hand-off waits (LLA_TC_POLL): 2, the default, polls with a nap between polls (the
+  // MMA issuers, usually a tile or two ahead of the epilogue, LLA_TC_NAP ns, 1000; the
+  // epilogue LLA_TC_ENAP ns, 64); 1 polls; 0 suspends.  Measured on the 21.3x workload
+  // over many B200s: polling took 537-545 us per call on some and 570-632 us on others
+  // (same code, same clocks), napping 561-570 us on both kinds.
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.enap_ns)
            : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
@@ -2952,7 +2952,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   const CUtensorMapSwizzle swz = p.box_k == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
-  p.poll = env_int("LLA_TC_POLL", 1);
+  p.poll = env_int("LLA_TC_POLL", 2);
   p.nap_ns = (uint32_t)env_int("LLA_TC_NAP", 1000);
   p.enap_ns = (uint32_t)env_int("LLA_TC_ENAP", 64);
   p.lat_hk = (int)a.lat_head_k;
