@@ -72,6 +72,7 @@ struct TcParams {
   int nbuf_b, n_p, m_v;
   int poll;                                  // per-head hand-offs poll instead of suspending
   uint32_t nap_ns, enap_ns;                  // naps between polls: MMA issuers, epilogue
+  uint32_t spins;                            // polls before the first nap
   // fused split combine (per-head kernel): the CTA that finishes a group's last split
   // merges the splits, adds the in-flight token and up-projects with W_up,v
   const float* q;                            // [B][H][d]
@@ -1811,12 +1812,12 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   // over many B200s: polling took 537-545 us per call on some and 570-632 us on others
   // (same code, same clocks), napping 561-570 us on both kinds.
   auto wait = [&](uint64_t* bar, uint32_t parity) {
-    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.enap_ns)
+    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.enap_ns, p.spins)
            : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
                        : mbar_wait(bar, parity, abort_flag);
   };
   auto wait_mma = [&](uint64_t* bar, uint32_t parity) {
-    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.nap_ns)
+    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.nap_ns, p.spins)
            : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
                        : mbar_wait(bar, parity, abort_flag);
   };
@@ -2955,6 +2956,7 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
   p.poll = env_int("LLA_TC_POLL", 2);
   p.nap_ns = (uint32_t)env_int("LLA_TC_NAP", 1000);
   p.enap_ns = (uint32_t)env_int("LLA_TC_ENAP", 64);
+  p.spins = (uint32_t)env_int("LLA_TC_SPIN", 0);
   p.lat_hk = (int)a.lat_head_k;
   p.lat_hv = (int)a.lat_head_v;
   if (pl.fform) {

@@ -115,8 +115,11 @@ __device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity,
 // long takes few issue slots from the warps sharing its sub-partition while still
 // noticing the phase within about nap_ns.
 __device__ __forceinline__ bool mbar_wait_nap(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag, uint32_t nap_ns) {
+                                              volatile int* abort_flag, uint32_t nap_ns,
+                                              uint32_t spins = 0) {
   if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t i = 0; i < spins; ++i)      // a short spin first: most hand-offs are near
+    if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     __nanosleep(nap_ns);
