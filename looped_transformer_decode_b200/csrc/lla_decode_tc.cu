@@ -93,6 +93,11 @@ struct TcParams {
   // 3: 64-byte rows)
   uint32_t e_off, e_bytes, b_img_bytes;
   int ne, n_f, kswz_mask;
+  // phase table (phase-operand kernel): tile_p0[b][tile] is the position of the tile's
+  // first token when its tokens sit at consecutive positions inside the table, whose
+  // row p holds conj(e^{i p theta_i}) as bf16 pairs; -1 (or no table) otherwise
+  const int32_t* tile_p0;
+  int n_tiles_cap;                           // tiles per sequence: ceil(n_cap / 128)
   const float2* rope;    // [rope_max_pos][d/2]
   const int32_t* ctx_len;
   const int32_t* positions;
@@ -105,6 +110,14 @@ struct TcParams {
   // conj(e^{i 128 theta_i}): advances conj(e^{i p theta_i}) by one tile of positions
   float2 step[64];
 };
+
+// compile-time value passed to generic lambdas
+template <int V>
+struct IntTag {
+  static constexpr int value = V;
+};
+// how the phase-operand kernel's epilogue gets its phase tiles
+constexpr int kPhaseComputed = 0, kPhaseMixed = 1, kPhaseTable = 2;
 
 constexpr int kNoPos = -2147483647 - 1;       // raw position of a row past the context
 constexpr int kReseedTiles = 32;              // exact RoPE factors at least this often
@@ -309,6 +322,14 @@ __device__ __forceinline__ int cursor_pos(const TcParams& p, const TileCursor& c
   const int t0 = c.r.tok0 + c.k * kTile;
   if (row >= c.r.tok_end - t0) return kNoPos;
   return p.positions[(size_t)c.r.b * p.n_cap + t0 + row];
+}
+
+// Table mark of the cursor's tile: the position of its first token when the prep grid
+// found the tile's positions consecutive inside the phase table, else -1 (and -1
+// without a table or past the last tile).
+__device__ __forceinline__ int cursor_tp0(const TcParams& p, const TileCursor& c) {
+  if (!p.tile_p0 || !c.valid) return -1;
+  return __ldcg(p.tile_p0 + (size_t)c.r.b * p.n_tiles_cap + c.r.s * p.tps + c.k);
 }
 
 __device__ __forceinline__ int checked_pos(const TcParams& p, int pos) {
@@ -1694,22 +1715,57 @@ __global__ void __launch_bounds__(kThreads2, 1)
 // of n_f x 128 bytes; 16-byte chunk c of row n at chunk c ^ (n % 8)).  Row g r_k + m
 // is B_m of head g, rows G r_k + 2g and + 1 its bias M~ as bf16 hi and lo, the rest
 // zero.  One CTA of 128 threads per (h, b).
+//
+// With a phase table (table non-null) the grid also writes, from the fp32 RoPE table,
+// rows [0, t_rows) of the phase table: row p holds (cos p theta_i, -sin p theta_i) as
+// bf16 at entries (2i, 2i + 1), the row of E for a token at position p.  And CTA
+// (h, b) marks tiles h, h + H, ... of sequence b: tile_p0[b][k] is the position of
+// the tile's first token when every token of the tile within the context sits at that
+// position plus its offset in the tile and the tile's rows lie inside the table, else
+// -1; such a tile's E is rows p0 .. p0 + 127 of the table.
 template <int D>
 __global__ void __launch_bounds__(128) decode_prep_f_kernel(
     const float* __restrict__ q, const int32_t* __restrict__ q_pos, const float2* __restrict__ rope,
     int rope_max_pos, const float* __restrict__ wupk_t, const float* __restrict__ muk_t, float kappa,
     int H, int r_k, int G, int n_f, uint32_t img_bytes, unsigned char* __restrict__ ops,
-    int32_t* status, uint32_t* counters) {
+    int32_t* status, uint32_t* counters, const int32_t* __restrict__ positions,
+    const int32_t* __restrict__ ctx_len, int n_cap, int n_tiles_cap, int32_t* __restrict__ tile_p0,
+    uint32_t* __restrict__ table, int t_rows) {
   constexpr int HALF = D / 2;
   constexpr int EBLK = D / 64;
   // the partial kernel may start its prologue and latent loads now; it waits for
-  // this grid before it reads the images or the counter
+  // this grid before it reads the images, the table, the tile marks or the counter
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float2 qc[HALF];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int g = h % G;
   if (counters && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0)
     counters[(size_t)gridDim.y * H] = 0u;
+  if (table) {
+    const size_t n_pairs = (size_t)t_rows * HALF;
+    const size_t stride = (size_t)gridDim.x * gridDim.y * 128;
+    for (size_t idx = ((size_t)b * gridDim.x + h) * 128 + tid; idx < n_pairs; idx += stride) {
+      const float2 e = rope[idx];   // (cos, sin) of pair idx % HALF at position idx / HALF
+      const __nv_bfloat162 v = __floats2bfloat162_rn(e.x, -e.y);
+      uint32_t u;
+      memcpy(&u, &v, 4);
+      table[idx] = u;
+    }
+    int n = ctx_len[b];
+    n = n < 0 ? 0 : (n > n_cap ? n_cap : n);   // the decode kernel flags a bad length
+    for (int k = h; k < n_tiles_cap; k += H) {
+      const int t0 = k * kTile, cnt = min(kTile, n - t0);
+      int ok = 0, p0 = -1;
+      if (cnt > 0) {
+        const int32_t* pr = positions + (size_t)b * n_cap + t0;
+        p0 = pr[0];
+        ok = tid >= cnt || (uint32_t)pr[tid] == (uint32_t)p0 + (uint32_t)tid;
+        ok = ok && p0 >= 0 && p0 <= t_rows - cnt;
+      }
+      ok = __syncthreads_and(ok);
+      if (tid == 0) tile_p0[(size_t)b * n_tiles_cap + k] = ok ? p0 : -1;
+    }
+  }
   int qp = q_pos[b];
   if (qp < 0 || qp >= rope_max_pos) {
     if (tid == 0 && h == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
@@ -1780,7 +1836,8 @@ constexpr int kVProdWarpF = 2 + kEpiWarpsF, kVMmaWarpF = 3 + kEpiWarpsF;
 template <int D, int KP, bool FUSE>
 __global__ void __launch_bounds__(kThreadsF, 1)
     decode_tcf_kernel(const __grid_constant__ CUtensorMap map_k,
-                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ TcParams p) {
+                      const __grid_constant__ CUtensorMap map_v,
+                      const __grid_constant__ CUtensorMap map_e, const __grid_constant__ TcParams p) {
   constexpr int G = kGF;
   constexpr int WG_PAIRS = D / 2 / kEpiWGF;  // RoPE pairs of a token row each warpgroup writes
   constexpr uint32_t NACC = 3;               // F buffers in TMEM
@@ -1801,6 +1858,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   uint64_t* pfull = bempty + 2;          // [2] softmax weights written
   uint64_t* pempty = pfull + 2;          // [2] V MMA done with the weights buffer
   uint64_t* drain = pempty + 2;          // [2] each MMA issuer's last MMAs completed
+  uint64_t* etx = drain + 2;             // [2] phase tile's table copy landed (or none issued)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
 
@@ -1844,6 +1902,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(&etx[0], 1);
+    mbar_init(&etx[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1967,7 +2027,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int k = 0; k < r.ntiles; ++k, ++it, ra.next(NACC)) {
           const uint32_t e = it & 1u, eph = (it >> 1) & 1u;     // two phase buffers
           const uint32_t acc = ra.slot, aph = ra.phase;
-          if (!wait_mma(&efull[e], eph) || !wait_mma(&tempty[acc], aph ^ 1u)) {
+          if (!wait_mma(&efull[e], eph) || !wait_mma(&etx[e], eph) ||
+              !wait_mma(&tempty[acc], aph ^ 1u)) {
             ok = false;
             break;
           }
@@ -2035,15 +2096,46 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     float* olat = reinterpret_cast<float*>(sm + p.comb_off);   // [128]: lane g r_v + m
     float* misc = olat + 128;   // [64]: m per head [0, G), q . k_self partials [8, 8 + 4G)
 
+    // Which of this CTA's tiles take their phase rows from the table (the marks are
+    // the prep grid's output).  The epilogue below is compiled three times: every
+    // phase tile computed (kPhaseComputed), per tile as marked (kPhaseMixed), every
+    // one copied from the table (kPhaseTable, without the RoPE factors' state).
+    int phase_mode = kPhaseComputed;
+    if (p.tile_p0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int hit = 0, miss = 0;
+      for (int item = blockIdx.x + (et >> 5) * gridDim.x; item < p.n_items;
+           item += kEpiWarpsF * gridDim.x) {
+        const ItemRange r = item_range(p, ctx_s, item, false);
+        for (int k = lane; k < r.ntiles; k += 32) {
+          const int m = __ldcg(p.tile_p0 + (size_t)r.b * p.n_tiles_cap + r.s * p.tps + k);
+          hit |= m >= 0;
+          miss |= m < 0;
+        }
+      }
+      const bool any_hit = epi_barrier_or_n<kEpiThreadsF>(hit) != 0;
+      const bool any_miss = epi_barrier_or_n<kEpiThreadsF>(miss) != 0;
+      phase_mode = !any_hit ? kPhaseComputed : (any_miss ? kPhaseMixed : kPhaseTable);
+    }
+    auto epilogue = [&](auto mode_tag) {
+    constexpr int MODE = decltype(mode_tag)::value;
+    // who needs the marks: every thread when tiles differ, the copying thread otherwise
+    const bool need_mark = MODE == kPhaseMixed || (MODE == kPhaseTable && et == 0);
+
     // Phase tiles: the RoPE factors conj(e^{i p theta_i}) of this warpgroup's pairs at
     // this thread's token row of the last tile written, advanced by one complex
     // product when the next tile's token sits a tile further on (as in
     // decode_tc_kernel), and a cursor over the tiles still to write.  The position of
-    // the next tile to write is loaded one tile before it is used.
+    // the next tile to write is loaded one tile before it is used, and so is its table
+    // mark: a tile whose tokens sit at consecutive positions inside the phase table
+    // is copied from the table's rows instead (one thread issues the copy).
     TileCursor ec;
     cursor_first(p, ctx_s, ec);
     bool e_more = ec.valid;                   // a phase tile is left to write
-    int pos_pref = cursor_pos(p, ec, row);    // its raw position at this thread's row
+    // its raw position at this thread's row, and its first position in the table (or -1)
+    int pos_pref = MODE == kPhaseTable ? kNoPos : cursor_pos(p, ec, row);
+    int tp_pref = need_mark ? cursor_tp0(p, ec) : -1;
+    int tp_cur = -1;                          // the same for the tile being written
     cursor_next(p, ctx_s, ec);
     float2 ef[WG_PAIRS];
     int pos_cur = kNoPos, run = 0;
@@ -2076,16 +2168,35 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     // The factors of the next phase tile (its position was loaded a tile ago), and the
     // position of the one after it.
     auto advance_e = [&]() {
-      advance_rope(pos_pref);
+      tp_cur = tp_pref;
+      if (MODE == kPhaseComputed || (MODE == kPhaseMixed && tp_cur < 0))
+        advance_rope(pos_pref);
+      else
+        pos_cur = kNoPos;                     // factors not kept: the next computed tile reseeds
       e_more = ec.valid;
-      pos_pref = cursor_pos(p, ec, row);      // used by the next advance
+      if (MODE != kPhaseTable) pos_pref = cursor_pos(p, ec, row);   // used by the next advance
+      if (need_mark) tp_pref = cursor_tp0(p, ec);
       cursor_next(p, ctx_s, ec);
     };
     // This thread's row of that tile into buffer ie % ne: entries (2i, 2i + 1) =
     // (cos, -sin) of pair i, 128-byte swizzled K-major rows.  The caller fences and
-    // arrives on efull[(ie - 1) % ne].
+    // arrives on efull[(ie - 1) % ne].  A table tile is one copy of D / 64 boxes of 64
+    // columns x 128 rows (rows past the table read as zeros) onto etx, which the F MMA
+    // issuer also waits for; a computed tile arrives on etx without a copy.
     auto store_e = [&]() {
-      unsigned char* eb = sm + p.e_off + (ie & 1u) * p.e_bytes;
+      const uint32_t eb_i = ie & 1u;
+      unsigned char* eb = sm + p.e_off + eb_i * p.e_bytes;
+      if (MODE == kPhaseTable || (MODE == kPhaseMixed && tp_cur >= 0)) {
+        if (et == 0) {
+          mbar_arrive_expect_tx(&etx[eb_i], (uint32_t)(kTile * D * 2));
+#pragma unroll
+          for (int blk = 0; blk < D / 64; ++blk)
+            tma_load_3d(eb + blk * (kTile * 128), &map_e, &etx[eb_i], blk * 64, tp_cur, 0);
+        }
+        ++ie;
+        return;
+      }
+      if (et == 0) mbar_arrive(&etx[eb_i]);
 #pragma unroll
       for (int c = 0; c < WG_PAIRS / 4; ++c) {
         const int pair0 = wgi * WG_PAIRS + c * 4;
@@ -2337,6 +2448,23 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       }
       named_barrier(1, kEpiThreadsF);           // scratch free for the next item
     }
+    if (MODE != kPhaseComputed && et == 0 && (aborted || *abort_flag)) {
+      // Drain: wait (bounded) for the table copies this thread issued (the last two
+      // phase tiles; a computed tile's etx phase is already complete).
+      for (uint32_t j = ie > 2u ? ie - 2u : 0u; j < ie; ++j) {
+        const unsigned long long t0 = global_timer_ns();
+        while (!mbar_try_wait(&etx[j & 1u], (j >> 1) & 1u) &&
+               global_timer_ns() - t0 < kWaitTimeoutNs) {
+        }
+      }
+    }
+    };   // epilogue
+    if (phase_mode == kPhaseTable)
+      epilogue(IntTag<kPhaseTable>{});
+    else if (phase_mode == kPhaseMixed)
+      epilogue(IntTag<kPhaseMixed>{});
+    else
+      epilogue(IntTag<kPhaseComputed>{});
   }
 
   tc_fence_before();
@@ -2550,10 +2678,26 @@ uint32_t tcf_layout(TcParams& p, int D, int G, int nst, int nst_v, int nbuf_b, i
   p.rope_off = o;
   o += 64 * 8 * 2;
   p.bar_off = o;
-  o += (2 * nst + 2 * nst_v + 18) * 8;
+  o += (2 * nst + 2 * nst_v + 20) * 8;
   p.misc_off = o;
   o += 16;
   return o + 1024;
+}
+
+// Workspace of the phase-operand path, in this order: the items' operand images
+// ([B][HG] of n_f x d bf16), the phase table (rows [0, n_tiles 128 + 128) of d bf16,
+// 1024-byte aligned) and the tile marks ([B][n_tiles] int32).
+constexpr size_t kAlignTable = 1024;
+size_t tcf_images_bytes(int B, int HG, int n_f, int d) { return (size_t)B * HG * n_f * d * 2; }
+size_t tcf_table_off(int B, int HG, int n_f, int d) {
+  return (tcf_images_bytes(B, HG, n_f, d) + kAlignTable - 1) / kAlignTable * kAlignTable;
+}
+int tcf_table_rows_cap(int n_cap) { return (n_cap + kTile - 1) / kTile * kTile + kTile; }
+size_t tcf_marks_off(int B, int HG, int n_f, int d, int n_cap) {
+  return tcf_table_off(B, HG, n_f, d) + (size_t)tcf_table_rows_cap(n_cap) * d * 2;
+}
+size_t tcf_ops_bytes(int B, int HG, int n_f, int d, int n_cap) {
+  return tcf_marks_off(B, HG, n_f, d, n_cap) + (size_t)B * ((n_cap + kTile - 1) / kTile) * 4;
 }
 
 // Whether the phase-operand kernel takes the shape: per head, RoPE over the whole
@@ -2725,7 +2869,7 @@ TcPlan tc_plan(const lla_cfg& c, int B, int n_cap) {
   pl.tps = (n_tiles + best_s - 1) / best_s;
   pl.S = (n_tiles + pl.tps - 1) / pl.tps;
   const size_t K_pad = (c.r_k + 15) / 16 * 16;
-  pl.ops_bytes = pl.fform ? (size_t)B * (c.H / pl.G) * ((size_t)pl.G * c.r_k + 16) * c.d_head * 2
+  pl.ops_bytes = pl.fform ? tcf_ops_bytes(B, c.H / pl.G, pl.G * c.r_k + 16, c.d_head, n_cap)
                           : (size_t)B * c.H * ((size_t)D * K_pad * 2 + (size_t)D * 32);
   pl.nope = nope;
   pl.ok = true;
@@ -2795,9 +2939,9 @@ cudaError_t launch_tc_nope(int G, bool shared, const CUtensorMap& mk, const CUte
 }
 
 template <int D, int KP>
-cudaError_t launch_tcf_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcParams& p,
-                         uint32_t smem, int grid, cudaStream_t s) {
-  void (*kern)(CUtensorMap, CUtensorMap, TcParams) =
+cudaError_t launch_tcf_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& me,
+                         const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, TcParams) =
       p.fuse_combine ? decode_tcf_kernel<D, KP, true> : decode_tcf_kernel<D, KP, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -2813,29 +2957,35 @@ cudaError_t launch_tcf_t(const CUtensorMap& mk, const CUtensorMap& mv, const TcP
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
+  return cudaLaunchKernelEx(&cfg, kern, mk, mv, me, p);
 }
 
 cudaError_t launch_tcf(int D, int KP, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const TcParams& p, uint32_t smem, int grid, cudaStream_t s) {
-  if (D == 128 && KP == 16) return launch_tcf_t<128, 16>(mk, mv, p, smem, grid, s);
-  if (D == 128 && KP == 32) return launch_tcf_t<128, 32>(mk, mv, p, smem, grid, s);
-  if (D == 64 && KP == 16) return launch_tcf_t<64, 16>(mk, mv, p, smem, grid, s);
-  if (D == 64 && KP == 32) return launch_tcf_t<64, 32>(mk, mv, p, smem, grid, s);
+                       const CUtensorMap& me, const TcParams& p, uint32_t smem, int grid,
+                       cudaStream_t s) {
+  if (D == 128 && KP == 16) return launch_tcf_t<128, 16>(mk, mv, me, p, smem, grid, s);
+  if (D == 128 && KP == 32) return launch_tcf_t<128, 32>(mk, mv, me, p, smem, grid, s);
+  if (D == 64 && KP == 16) return launch_tcf_t<64, 16>(mk, mv, me, p, smem, grid, s);
+  if (D == 64 && KP == 32) return launch_tcf_t<64, 32>(mk, mv, me, p, smem, grid, s);
   return cudaErrorNotSupported;
 }
 
-cudaError_t launch_prep_f(const DecodeArgs& a, const TcParams& p, int G, cudaStream_t s) {
+// table / t_rows: the phase table to write and its rows (null: no table, no marks)
+cudaError_t launch_prep_f(const DecodeArgs& a, const TcParams& p, int G, uint32_t* table,
+                          int t_rows, cudaStream_t s) {
   dim3 grid((unsigned)a.H, (unsigned)a.B);
   unsigned char* ob = const_cast<unsigned char*>(p.ops_b);
+  int32_t* marks = const_cast<int32_t*>(p.tile_p0);
   if (a.d == 128)
-    decode_prep_f_kernel<128><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t,
-                                                   a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
-                                                   p.b_img_bytes, ob, a.status, a.counters);
+    decode_prep_f_kernel<128><<<grid, 128, 0, s>>>(
+        a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
+        p.b_img_bytes, ob, a.status, a.counters, a.positions, a.ctx_len, a.n_cap, p.n_tiles_cap,
+        marks, table, t_rows);
   else if (a.d == 64)
-    decode_prep_f_kernel<64><<<grid, 128, 0, s>>>(a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t,
-                                                  a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
-                                                  p.b_img_bytes, ob, a.status, a.counters);
+    decode_prep_f_kernel<64><<<grid, 128, 0, s>>>(
+        a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
+        p.b_img_bytes, ob, a.status, a.counters, a.positions, a.ctx_len, a.n_cap, p.n_tiles_cap,
+        marks, table, t_rows);
   else
     return cudaErrorNotSupported;
   return cudaGetLastError();
@@ -2965,11 +3115,27 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
     if (!make_map(&mk, a.ck, (int)a.lat_tok_k, a.n_cap, a.B, p.box_k, swz) ||
         !make_map(&mv, a.cv, (int)a.lat_tok_v, a.n_cap, a.B, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorNotSupported;
+    // Phase table (LLA_TCF_TABLE=0 leaves every phase tile computed): rows up to the
+    // cache's tile-rounded length plus one tile, within the RoPE table, and at least
+    // one tile of them
+    CUtensorMap me;
+    std::memset(&me, 0, sizeof(me));
+    uint32_t* table = nullptr;
+    const int t_rows = std::min(a.rope_max_pos, tcf_table_rows_cap(a.n_cap));
+    p.n_tiles_cap = (a.n_cap + kTile - 1) / kTile;
+    p.tile_p0 = nullptr;
+    if (env_int("LLA_TCF_TABLE", 1) != 0 && t_rows >= kTile) {
+      const int HG = a.H / pl.G;
+      table = reinterpret_cast<uint32_t*>(a.ops + tcf_table_off(a.B, HG, p.n_f, a.d));
+      p.tile_p0 = reinterpret_cast<const int32_t*>(a.ops + tcf_marks_off(a.B, HG, p.n_f, a.d, a.n_cap));
+      if (!make_map(&me, table, a.d, t_rows, 1, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorNotSupported;
+    }
     const int sms = sm_count();
-    cudaError_t pe = launch_prep_f(a, p, pl.G, s);
+    cudaError_t pe = launch_prep_f(a, p, pl.G, table, t_rows, s);
     if (pe != cudaSuccess) return pe;
     const int grid = p.n_items < sms ? p.n_items : sms;
-    cudaError_t e = launch_tcf(a.d, a.r_k, mk, mv, p, smem, grid, s);
+    cudaError_t e = launch_tcf(a.d, a.r_k, mk, mv, me, p, smem, grid, s);
     if (e == cudaSuccess && !p.fuse_combine) e = launch_combine(a, s);
     return e;
   }

@@ -167,8 +167,10 @@ def test_forced_split_count_is_clamped(monkeypatch):
 def test_phase_operand_kernel_workspace():
     """Per-head shapes with r_k in {16, 32} and r_v = 32 run on the phase-operand
     kernel, whose operand images are one [4 r_k + 16, d] bf16 image per (sequence,
-    group of four heads); LLA_TC_FORM=u keeps them on the per-head kernel, whose
-    images are per (sequence, head)."""
+    group of four heads), followed (1024-byte aligned) by the phase table, bf16 rows
+    of d entries for positions below the tile-rounded cache length plus one tile,
+    and one int32 table mark per (sequence, tile); LLA_TC_FORM=u keeps them on the
+    per-head kernel, whose images are per (sequence, head)."""
     import os
     cfg = lla.Cfg(4, 16, 128, 16, 32)
     c = ctypes.byref(cfg.c())
@@ -180,6 +182,10 @@ def test_phase_operand_kernel_workspace():
     finally:
         del os.environ["LLA_TC_FORM"]
     img_f = B * (16 // 4) * (4 * 16 + 16) * 128 * 2
+    n_tiles = -(-n // 128)
+    table = (n_tiles * 128 + 128) * 128 * 2
+    marks = B * n_tiles * 4
+    assert img_f % 1024 == 0
     img_u = B * 16 * (128 * 16 * 2 + 128 * 32)
-    assert ws_u - ws_f == img_u - img_f
+    assert ws_u - ws_f == img_u - (img_f + table + marks)
     assert lla.decode_launches(cfg, B, n) == 2

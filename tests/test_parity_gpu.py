@@ -235,6 +235,42 @@ def test_per_head_kernel_on_phase_operand_shapes(spec, monkeypatch):
     assert lla.decode_status(dev.ws) == 0
 
 
+def _phase_table_case(cfg, seed):
+    """One call whose sequences take phase tiles from the table, computed, or both:
+    consecutive positions from 0; offset by 100 (every tile inside the table's
+    tile-rounded cache length plus one tile, 768 rows); offset by 200 (the last tile
+    runs past those rows); a gap of 5 inside tile 2 (that tile computed, the next
+    ones consecutive again); arbitrary positions; a ragged and an empty context."""
+    B, n_cap = 7, 600
+    case = decode_case(cfg, B, n_cap, seed=seed, ctx_len=[600, 600, 600, 600, 600, 130, 0])
+    pos = np.tile(np.arange(n_cap), (B, 1))
+    pos[1] += 100
+    pos[2] += 200
+    pos[3, 300:] += 5
+    pos[4] = synth.rng(seed + 1).permutation(4 * n_cap)[:n_cap]
+    case.positions = pos
+    case.q_pos = np.array([600, 700, 800, 605, 2400, 130, 0])
+    return case
+
+
+@pytest.mark.parametrize("cfg", [O.Cfg(4, 4, 128, 16, 32), O.Cfg(4, 8, 64, 32, 32)],
+                         ids=lambda c: f"H{c.H}d{c.d}r{c.r_k}")
+def test_phase_table_and_computed_tiles_match_oracle(cfg, monkeypatch):
+    """The phase-operand kernel copies a tile's phase rows from the phase table when
+    the tile's positions are consecutive inside it and computes them otherwise
+    (LLA_TCF_TABLE=0: always); both against the oracle on the same call."""
+    case = _phase_table_case(cfg, seed=900 + cfg.d)
+    dev = DeviceCase(case)
+    for mode in ("1", "0"):
+        monkeypatch.setenv("LLA_TCF_TABLE", mode)
+        for t in (0, cfg.T - 1):
+            got = dev.decode(t)
+            assert np.isfinite(got).all(), (mode, t)
+            err = rel_err(got, expected(case, t))
+            assert err.max() <= ATTN_TOL, (mode, t, err.max())
+        assert lla.decode_status(dev.ws) == 0
+
+
 NAN_TAIL = [
     (O.Cfg(4, 2, 128, 96, 160), 2, 300, [300, 190], "tensor_core"),     # per-head kernel
     (O.Cfg(4, 4, 128, 16, 32), 2, 300, [300, 190], "tensor_core"),      # phase-operand kernel
