@@ -1718,92 +1718,145 @@ __global__ void __launch_bounds__(kThreads2, 1)
 //
 // With a phase table (table non-null) the grid also writes, from the fp32 RoPE table,
 // rows [0, t_rows) of the phase table: row p holds (cos p theta_i, -sin p theta_i) as
-// bf16 at entries (2i, 2i + 1), the row of E for a token at position p.  And CTA
-// (h, b) marks tiles h, h + H, ... of sequence b: tile_p0[b][k] is the position of
-// the tile's first token when every token of the tile within the context sits at that
-// position plus its offset in the tile and the tile's rows lie inside the table, else
-// -1; such a tile's E is rows p0 .. p0 + 127 of the table.
-template <int D>
+// bf16 at entries (2i, 2i + 1), the row of E for a token at position p.  And warp w of
+// CTA (h, b) marks tiles 4h + w, 4h + w + 4H, ... of sequence b: tile_p0[b][k] is the
+// position of the tile's first token when every token of the tile within the context
+// sits at that position plus its offset in the tile and the tile's rows lie inside
+// the table, else -1; such a tile's E is rows p0 .. p0 + 127 of the table.
+//
+// Each CTA stages its head's W_up,k ([d][KP] fp32) and mu in shared memory with
+// coalesced 16-byte reads (every CTA of a head reads the same 8-16 KB from L2), and
+// every read that depends on nothing else (weights, query, q_pos, ctx_len, the first
+// tile's positions, a table row) is issued before the first wait.
+template <int D, int KP>
 __global__ void __launch_bounds__(128) decode_prep_f_kernel(
     const float* __restrict__ q, const int32_t* __restrict__ q_pos, const float2* __restrict__ rope,
     int rope_max_pos, const float* __restrict__ wupk_t, const float* __restrict__ muk_t, float kappa,
-    int H, int r_k, int G, int n_f, uint32_t img_bytes, unsigned char* __restrict__ ops,
-    int32_t* status, uint32_t* counters, const int32_t* __restrict__ positions,
-    const int32_t* __restrict__ ctx_len, int n_cap, int n_tiles_cap, int32_t* __restrict__ tile_p0,
-    uint32_t* __restrict__ table, int t_rows) {
+    int H, int G, int n_f, uint32_t img_bytes, unsigned char* __restrict__ ops, int32_t* status,
+    uint32_t* counters, const int32_t* __restrict__ positions, const int32_t* __restrict__ ctx_len,
+    int n_cap, int n_tiles_cap, int32_t* __restrict__ tile_p0, uint32_t* __restrict__ table,
+    int t_rows) {
   constexpr int HALF = D / 2;
   constexpr int EBLK = D / 64;
+  constexpr int WS = KP + 1;                     // padded row of the staged weights
+  constexpr int NW4 = D * KP / 4 / 128;          // 16-byte weight reads per thread
   // the partial kernel may start its prologue and latent loads now; it waits for
   // this grid before it reads the images, the table, the tile marks or the counter
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float2 qc[HALF];
+  __shared__ float ws[D * WS];
+  __shared__ float mus[D];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int g = h % G;
   if (counters && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0)
     counters[(size_t)gridDim.y * H] = 0u;
-  if (table) {
-    const size_t n_pairs = (size_t)t_rows * HALF;
-    const size_t stride = (size_t)gridDim.x * gridDim.y * 128;
-    for (size_t idx = ((size_t)b * gridDim.x + h) * 128 + tid; idx < n_pairs; idx += stride) {
-      const float2 e = rope[idx];   // (cos, sin) of pair idx % HALF at position idx / HALF
-      const __nv_bfloat162 v = __floats2bfloat162_rn(e.x, -e.y);
-      uint32_t u;
-      memcpy(&u, &v, 4);
-      table[idx] = u;
-    }
-    int n = ctx_len[b];
-    n = n < 0 ? 0 : (n > n_cap ? n_cap : n);   // the decode kernel flags a bad length
-    for (int k = h; k < n_tiles_cap; k += H) {
-      const int t0 = k * kTile, cnt = min(kTile, n - t0);
-      int ok = 0, p0 = -1;
-      if (cnt > 0) {
-        const int32_t* pr = positions + (size_t)b * n_cap + t0;
-        p0 = pr[0];
-        ok = tid >= cnt || (uint32_t)pr[tid] == (uint32_t)p0 + (uint32_t)tid;
-        ok = ok && p0 >= 0 && p0 <= t_rows - cnt;
-      }
-      ok = __syncthreads_and(ok);
-      if (tid == 0) tile_p0[(size_t)b * n_tiles_cap + k] = ok ? p0 : -1;
-    }
+
+  // ---- reads that depend on nothing else
+  const int qp_raw = q_pos[b];
+  const float* qh = q + ((size_t)b * H + h) * D;
+  float x0 = 0.f, x1 = 0.f;
+  if (tid < HALF) {
+    x0 = qh[tid];
+    x1 = qh[tid + HALF];
   }
-  int qp = q_pos[b];
+  const float4* W4 = reinterpret_cast<const float4*>(wupk_t + (size_t)h * D * KP);   // [d][KP]
+  float4 w4[NW4];
+#pragma unroll
+  for (int j = 0; j < NW4; ++j) w4[j] = W4[tid + 128 * j];
+  const float mu_v = tid < D ? muk_t[(size_t)h * D + tid] : 0.f;
+  const size_t n_pairs = table ? (size_t)t_rows * HALF : 0;
+  const size_t t_stride = (size_t)gridDim.x * gridDim.y * 128;
+  const size_t t_idx0 = ((size_t)b * gridDim.x + h) * 128 + tid;
+  float2 te = make_float2(0.f, 0.f);
+  if (t_idx0 < n_pairs) te = rope[t_idx0];      // (cos, sin) of pair idx % HALF at idx / HALF
+  const int k0 = 4 * h + warp;                  // this warp's first tile
+  int n = 0, pv[4] = {0, 0, 0, 0};              // lane l holds offsets 4l .. 4l + 3
+  auto load_tile = [&](int k) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int t = k * kTile + lane * 4 + e;
+      pv[e] = t < n_cap ? positions[(size_t)b * n_cap + t] : 0;
+    }
+  };
+  if (table) {
+    n = ctx_len[b];
+    if (k0 < n_tiles_cap) load_tile(k0);
+  }
+#pragma unroll
+  for (int j = 0; j < NW4; ++j) {
+    const int f = 4 * (tid + 128 * j), i = f / KP, m = f % KP;   // 4 | KP: one row
+    float* dst = ws + i * WS + m;
+    dst[0] = w4[j].x;
+    dst[1] = w4[j].y;
+    dst[2] = w4[j].z;
+    dst[3] = w4[j].w;
+  }
+  if (tid < D) mus[tid] = mu_v;
+
+  // ---- the query's RoPE factors (wait for q_pos)
+  int qp = qp_raw;
   if (qp < 0 || qp >= rope_max_pos) {
     if (tid == 0 && h == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
     qp = 0;
   }
-  const float* qh = q + ((size_t)b * H + h) * D;
-  for (int i = tid; i < HALF; i += 128) {
-    const float2 e = rope[(size_t)qp * HALF + i];
-    const float x0 = qh[i], x1 = qh[i + HALF];
-    qc[i] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
+  if (tid < HALF) {
+    const float2 e = rope[(size_t)qp * HALF + tid];
+    qc[tid] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
+  }
+
+  // ---- table rows and tile marks while those land
+  if (table) {
+    auto put = [&](size_t idx, float2 e) {
+      const __nv_bfloat162 v = __floats2bfloat162_rn(e.x, -e.y);
+      uint32_t u;
+      memcpy(&u, &v, 4);
+      table[idx] = u;
+    };
+    if (t_idx0 < n_pairs) put(t_idx0, te);
+    for (size_t idx = t_idx0 + t_stride; idx < n_pairs; idx += t_stride) put(idx, rope[idx]);
+    n = n < 0 ? 0 : (n > n_cap ? n_cap : n);   // the decode kernel flags a bad length
+    for (int k = k0; k < n_tiles_cap; k += 4 * H) {
+      if (k != k0) load_tile(k);
+      const int cnt = min(kTile, n - k * kTile);
+      const int p0 = __shfl_sync(0xffffffffu, pv[0], 0);
+      bool ok = cnt > 0 && p0 >= 0 && p0 <= t_rows - cnt;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int off = lane * 4 + e;
+        ok = ok && (off >= cnt || (uint32_t)pv[e] == (uint32_t)p0 + (uint32_t)off);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (lane == 0) tile_p0[(size_t)b * n_tiles_cap + k] = ok ? p0 : -1;
+    }
   }
   __syncthreads();
-  const float* W = wupk_t + (size_t)h * D * r_k;   // [d][r_k]
-  const float* mu = muk_t + (size_t)h * D;
+
+  // ---- the image rows: this head's KP rows (W_up,k), its two bias rows (mu), and
+  // (first head of the group) the zero rows that pad n_f; chunk idx is 16-byte chunk c
+  // of column block kb of local row lr
   unsigned char* img = ops + ((size_t)b * (H / G) + h / G) * img_bytes;
-  // this head's rows: its r_k rows, its two bias rows, and (first head of the group)
-  // the zero rows that pad n_f
-  const int pad0 = G * r_k + 2 * G;
-  const int rows = r_k + 2 + (g == 0 ? n_f - pad0 : 0);
+  const int pad0 = G * KP + 2 * G;
+  const int rows = KP + 2 + (g == 0 ? n_f - pad0 : 0);
   for (int idx = tid; idx < rows * EBLK * 8; idx += 128) {
     const int lr = idx / (EBLK * 8), kb = (idx >> 3) % EBLK, c = idx & 7;
-    const int n = lr < r_k ? g * r_k + lr
-                           : (lr < r_k + 2 ? G * r_k + 2 * g + (lr - r_k) : pad0 + (lr - r_k - 2));
+    const int nr = lr < KP ? g * KP + lr
+                           : (lr < KP + 2 ? G * KP + 2 * g + (lr - KP) : pad0 + (lr - KP - 2));
     __align__(16) __nv_bfloat16 v[8];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int i = kb * 32 + c * 4 + e;       // RoPE pair of entries 2e, 2e + 1
       const float2 z = qc[i];
       float re = 0.f, im = 0.f;
-      if (lr < r_k) {
-        const float wr = W[(size_t)i * r_k + lr], wi = W[(size_t)(i + HALF) * r_k + lr];
+      if (lr < KP) {
+        const float wr = ws[i * WS + lr], wi = ws[(i + HALF) * WS + lr];
         re = kappa * (z.x * wr + z.y * wi);
         im = kappa * (z.x * wi - z.y * wr);
-      } else if (lr < r_k + 2) {
-        const float mr = mu[i], mi = mu[i + HALF];
+      } else if (lr < KP + 2) {
+        const float mr = mus[i], mi = mus[i + HALF];
         re = kappa * (z.x * mr + z.y * mi);
         im = kappa * (z.x * mi - z.y * mr);
-        if (lr == r_k + 1) {   // lo row: what the bf16 hi row leaves
+        if (lr == KP + 1) {   // lo row: what the bf16 hi row leaves
           re -= __bfloat162float(__float2bfloat16_rn(re));
           im -= __bfloat162float(__float2bfloat16_rn(im));
         }
@@ -1811,7 +1864,7 @@ __global__ void __launch_bounds__(128) decode_prep_f_kernel(
       v[2 * e] = __float2bfloat16_rn(re);
       v[2 * e + 1] = __float2bfloat16_rn(im);
     }
-    *reinterpret_cast<uint4*>(img + (size_t)kb * n_f * 128 + (size_t)n * 128 + ((c ^ (n & 7)) << 4)) =
+    *reinterpret_cast<uint4*>(img + (size_t)kb * n_f * 128 + (size_t)nr * 128 + ((c ^ (nr & 7)) << 4)) =
         *reinterpret_cast<const uint4*>(v);
   }
 }
@@ -2976,18 +3029,22 @@ cudaError_t launch_prep_f(const DecodeArgs& a, const TcParams& p, int G, uint32_
   dim3 grid((unsigned)a.H, (unsigned)a.B);
   unsigned char* ob = const_cast<unsigned char*>(p.ops_b);
   int32_t* marks = const_cast<int32_t*>(p.tile_p0);
-  if (a.d == 128)
-    decode_prep_f_kernel<128><<<grid, 128, 0, s>>>(
-        a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
-        p.b_img_bytes, ob, a.status, a.counters, a.positions, a.ctx_len, a.n_cap, p.n_tiles_cap,
-        marks, table, t_rows);
-  else if (a.d == 64)
-    decode_prep_f_kernel<64><<<grid, 128, 0, s>>>(
-        a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, a.muk_t, a.kappa, a.H, a.r_k, G, p.n_f,
-        p.b_img_bytes, ob, a.status, a.counters, a.positions, a.ctx_len, a.n_cap, p.n_tiles_cap,
-        marks, table, t_rows);
+#define LLA_PREP_F(DD, KK)                                                                  \
+  decode_prep_f_kernel<DD, KK><<<grid, 128, 0, s>>>(                                        \
+      a.q, a.q_pos, a.rope, a.rope_max_pos, a.wupk_t, a.muk_t, a.kappa, a.H, G, p.n_f,        \
+      p.b_img_bytes, ob, a.status, a.counters, a.positions, a.ctx_len, a.n_cap, p.n_tiles_cap, \
+      marks, table, t_rows)
+  if (a.d == 128 && a.r_k == 16)
+    LLA_PREP_F(128, 16);
+  else if (a.d == 128 && a.r_k == 32)
+    LLA_PREP_F(128, 32);
+  else if (a.d == 64 && a.r_k == 16)
+    LLA_PREP_F(64, 16);
+  else if (a.d == 64 && a.r_k == 32)
+    LLA_PREP_F(64, 32);
   else
     return cudaErrorNotSupported;
+#undef LLA_PREP_F
   return cudaGetLastError();
 }
 
