@@ -72,6 +72,7 @@ struct TcParams {
   int nbuf_b, n_p, m_v;
   int poll;                                  // per-head hand-offs poll instead of suspending
   uint32_t nap_ns, enap_ns;                  // naps between polls: MMA issuers, epilogue
+  uint32_t cnap_ns;                          // MMA issuers of a CTA whose phase tiles are all computed
   uint32_t spins;                            // polls before the first nap
   // fused split combine (per-head kernel): the CTA that finishes a group's last split
   // merges the splits, adds the in-flight token and up-projects with W_up,v
@@ -1914,21 +1915,30 @@ __global__ void __launch_bounds__(kThreadsF, 1)
   uint64_t* etx = drain + 2;             // [2] phase tile's table copy landed (or none issued)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + p.misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + p.misc_off + 4);
+  // how this CTA gets its phase tiles (kPhase*), written by the epilogue before its
+  // first hand-off
+  volatile int* phase_mode_s = reinterpret_cast<volatile int*>(sm + p.misc_off + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int* ctx_s = p.B <= kCtxCache ? reinterpret_cast<const int*>(sm + p.ctx_off) : nullptr;
   // Hand-off waits (LLA_TC_POLL): 2, the default, polls with a nap between polls (the
-  // MMA issuers, usually a tile or two ahead of the epilogue, LLA_TC_NAP ns, 1000; the
-  // epilogue LLA_TC_ENAP ns, 64); 1 polls; 0 suspends.  Measured on the 21.3x workload
-  // over many B200s: polling took 537-545 us per call on some and 570-632 us on others
-  // (same code, same clocks), napping 561-570 us on both kinds.
+  // epilogue LLA_TC_ENAP ns, 64; the MMA issuers LLA_TC_NAP ns, 150, in a CTA with
+  // table tiles, LLA_TC_CNAP ns, 1000, in one without, known after their first
+  // hand-off); 1 polls; 0 suspends.  Measured on the 21.3x workload: with every phase
+  // tile computed, polling took 537-545 us per call on some B200s and 570-632 us on
+  // others (same code, same clocks), napping 561-570 us on both kinds, and an MMA nap
+  // of 150 ns 552 us against 540 us at 1000 ns; with table tiles the F MMA issuer also
+  // waits for the tile's copy, and MMA naps of 0-300 ns took 347-351 us per call
+  // against 369 us at 1000 ns, while polling everywhere took 425 us.
+  uint32_t mma_nap = p.nap_ns;
+  auto set_mma_nap = [&]() { mma_nap = *phase_mode_s == kPhaseComputed ? p.cnap_ns : p.nap_ns; };
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.enap_ns, p.spins)
            : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
                        : mbar_wait(bar, parity, abort_flag);
   };
   auto wait_mma = [&](uint64_t* bar, uint32_t parity) {
-    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, p.nap_ns, p.spins)
+    return p.poll == 2 ? mbar_wait_nap(bar, parity, abort_flag, mma_nap, p.spins)
            : p.poll    ? mbar_wait_poll(bar, parity, abort_flag)
                        : mbar_wait(bar, parity, abort_flag);
   };
@@ -2085,6 +2095,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             ok = false;
             break;
           }
+          if (it == 0) set_mma_nap();
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + acc * p.n_f;
           const uint32_t e_addr = e_base + e * p.e_bytes;
@@ -2122,6 +2133,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             ok = false;
             break;
           }
+          if (it == 0) set_mma_nap();
           tc_fence_after();
           const uint32_t a_addr = smem_addr(sm + p.stv_off + vs * p.stv_bytes);
           const uint32_t b_addr = p_base + pb * 4096u;
@@ -2170,6 +2182,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       const bool any_miss = epi_barrier_or_n<kEpiThreadsF>(miss) != 0;
       phase_mode = !any_hit ? kPhaseComputed : (any_miss ? kPhaseMixed : kPhaseTable);
     }
+    if (et == 0) *phase_mode_s = phase_mode;   // before its first arrival on efull
     auto epilogue = [&](auto mode_tag) {
     constexpr int MODE = decltype(mode_tag)::value;
     // who needs the marks: every thread when tiles differ, the copying thread otherwise
@@ -3161,7 +3174,8 @@ cudaError_t launch_decode_tc(const lla_cfg& c, const DecodeArgs& a, cudaStream_t
                                  : p.box_k == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   p.poll = env_int("LLA_TC_POLL", 2);
-  p.nap_ns = (uint32_t)env_int("LLA_TC_NAP", 1000);
+  p.nap_ns = (uint32_t)env_int("LLA_TC_NAP", 150);
+  p.cnap_ns = (uint32_t)env_int("LLA_TC_CNAP", 1000);
   p.enap_ns = (uint32_t)env_int("LLA_TC_ENAP", 64);
   p.spins = (uint32_t)env_int("LLA_TC_SPIN", 0);
   p.lat_hk = (int)a.lat_head_k;
