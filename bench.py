@@ -41,7 +41,7 @@ METRIC = "LLA decode-attention HBM GB/s (% of peak) and ctx-tokens/s per loop st
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of the
 # current kernels (profiles/); a workload without a capture of the current code reports null.
 NCU_TRAFFIC = {"perhead_4x_T4_H16_d128_r96_160_B8_n4096": 277.01e6,
-               "perhead_21x_T4_H16_d128_r16_32_B256_n4096_L24": 1650.84e6,
+               "perhead_21x_T4_H16_d128_r16_32_B256_n4096_L24": 1650.94e6,
                "lla2d_T4_H16_d128_r64_128_B512_n4096": 1008.05e6,
                # encode (the dominant kernel): a 32768-token capture scaled by 16 tokens-wise
                "deeploop_32x_T32_H8_d96_r64_128_B16_n32768": 55.24e9}
