@@ -366,6 +366,30 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
   // kernel runs first)
   if (counters && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0)
     counters[(size_t)gridDim.y * H] = 0u;
+  // This thread's first image chunk and first bias chunk need nothing from the query:
+  // their W_up,k and mu values are read before the query's RoPE factors (which wait
+  // for q_pos), so the two reads overlap.
+  const float* W = wupk_t + (size_t)h * d_full * r_k;  // [d][r_k]
+  const float* mu = muk_t + (size_t)h * d_full;
+  const int chunks = D * K_pad / 8;
+  const int c_first = blockIdx.z * blockDim.x + tid;
+  float w_first[16];
+  if (c_first < chunks) {
+    const int n = (c_first / K_pad) * 8 + (c_first & 7), k0 = ((c_first >> 3) % (K_pad / 8)) * 8;
+    const int i = n >> 1;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const bool in = k0 + e < r_k;
+      w_first[2 * e] = in ? W[(size_t)i * r_k + k0 + e] : 0.f;
+      w_first[2 * e + 1] = in ? W[(size_t)(i + HALF) * r_k + k0 + e] : 0.f;
+    }
+  }
+  float mu_first[2] = {0.f, 0.f};
+  if (c_first < D * 2 && ((c_first >> 3) & 1) == 0) {
+    const int i = ((c_first >> 4) * 8 + (c_first & 7)) >> 1;
+    mu_first[0] = mu[i];
+    mu_first[1] = mu[i + HALF];
+  }
   int qp = q_pos[b];
   if (qp < 0 || qp >= rope_max_pos) {
     if (tid == 0 && h == 0 && blockIdx.z == 0) atomicOr(status, LLA_STATUS_POSITION_RANGE);
@@ -378,12 +402,10 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
     qc[i] = make_float2(x0 * e.x - x1 * e.y, x0 * e.y + x1 * e.x);
   }
   __syncthreads();
-  const float* W = wupk_t + (size_t)h * d_full * r_k;  // [d][r_k]
   unsigned char* img = ops_b + ((size_t)b * H + h) * (size_t)NS * K_pad * 2;
   // One 16-byte chunk (8 consecutive K values of one row n) per iteration; rows < D
   // here, the 16 NoPE rows (decoupled RoPE) below.
-  const int chunks = D * K_pad / 8;
-  for (int c = blockIdx.z * blockDim.x + tid; c < chunks; c += gridDim.z * blockDim.x) {
+  for (int c = c_first; c < chunks; c += gridDim.z * blockDim.x) {
     const int n = (c / K_pad) * 8 + (c & 7);
     const int k0 = ((c >> 3) % (K_pad / 8)) * 8;
     __align__(16) __nv_bfloat16 v[8];
@@ -394,7 +416,8 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
       const int k = k0 + e;
       float val = 0.f;
       if (k < r_k) {
-        const float wr = W[(size_t)i * r_k + k], wi = W[(size_t)(i + HALF) * r_k + k];
+        const float wr = c == c_first ? w_first[2 * e] : W[(size_t)i * r_k + k];
+        const float wi = c == c_first ? w_first[2 * e + 1] : W[(size_t)(i + HALF) * r_k + k];
         val = (n & 1) ? kappa * (z.x * wi - z.y * wr) : kappa * (z.x * wr + z.y * wi);
       }
       v[e] = __float2bfloat16_rn(val);
@@ -444,8 +467,7 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
   // Bias tile image [D x 16]: chunk c covers row n = (c / 2 / 8) * 8 + c % 8 ... laid out as
   // core matrices (n / 8, k / 8) at (n / 8) * 256 + (k / 8) * 128 + (n % 8) * 16.
   unsigned char* bimg = ops_bias + ((size_t)b * H + h) * (size_t)NS * 32;
-  const float* mu = muk_t + (size_t)h * d_full;
-  for (int c = blockIdx.z * blockDim.x + tid; c < D * 2; c += gridDim.z * blockDim.x) {
+  for (int c = c_first; c < D * 2; c += gridDim.z * blockDim.x) {
     const int n = (c >> 4) * 8 + (c & 7);
     const int kc = (c >> 3) & 1;
     __align__(16) __nv_bfloat16 v[8];
@@ -454,7 +476,8 @@ __global__ void __launch_bounds__(128) decode_prep_kernel(
     if (kc == 0) {
       const int i = n >> 1;
       const float2 z = qc[i];
-      const float mr = mu[i], mi = mu[i + HALF];
+      const float mr = c == c_first ? mu_first[0] : mu[i];
+      const float mi = c == c_first ? mu_first[1] : mu[i + HALF];
       const float val = (n & 1) ? kappa * (z.x * mi - z.y * mr) : kappa * (z.x * mr + z.y * mi);
       v[0] = __float2bfloat16_rn(val);
       v[1] = __float2bfloat16_rn(val - __bfloat162float(v[0]));
