@@ -189,3 +189,15 @@ def test_phase_operand_kernel_workspace():
     img_u = B * 16 * (128 * 16 * 2 + 128 * 32)
     assert ws_u - ws_f == img_u - (img_f + table + marks)
     assert lla.decode_launches(cfg, B, n) == 2
+
+
+def test_phase_table_switch_keeps_the_workspace_size(monkeypatch):
+    """The phase table and tile marks are always reserved: LLA_TCF_TABLE only decides
+    whether a call uses them, so a workspace sized once serves either setting."""
+    cfg = lla.Cfg(4, 16, 128, 16, 32)
+    c = ctypes.byref(cfg.c())
+    for B, n in ((256, 4096), (3, 300), (1, 1)):
+        monkeypatch.setenv("LLA_TCF_TABLE", "1")
+        on = lla.lib.lla_decode_workspace_bytes(c, B, n)
+        monkeypatch.setenv("LLA_TCF_TABLE", "0")
+        assert lla.lib.lla_decode_workspace_bytes(c, B, n) == on
